@@ -1,0 +1,372 @@
+#!/usr/bin/env python3
+"""Bench of the quantized gated delta-rule decode step (libsq on B200).
+
+One step = one call of the whole hot path (sq_decode_step: unpack, gated delta update, output,
+dual-axis refit, requantize and repack in place) over one batch of synthetic requests. The
+default workload is the GDN-style layer: 64 requests x 32 heads, d_k = d_v = 128, per-head
+widths {4, 6, 8} (mean 6) plus 2 fp16 pivot heads, bf16 q/k/v.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload gdn|kda|pool]
+                    [--impl ours|reference]
+
+Prints one JSON line (rank 0). Multi-GPU: launched by torchrun, one process per GPU, each rank
+decoding its own requests (weak scaling, no collective on the data path); times are device
+times (CUDA events) and the max over ranks is reported. The reference arm (--impl reference)
+times the CPU oracle on a bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import glob
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from bit_recurrent_state_gated_b200 import dist  # noqa: E402
+from bit_recurrent_state_gated_b200 import workloads as W  # noqa: E402
+
+METRIC = "quantized delta-rule decode: request-steps/s and state HBM GB/s vs peak"
+UNIT = "request-steps/s"
+L2_FLUSH_BYTES = 256 << 20  # > 126 MB of L2
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="gdn", choices=["tiny", "gdn", "kda", "pool"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target CPU time of the oracle baseline sample")
+    return ap.parse_args()
+
+
+# ---- byte accounting ---------------------------------------------------------------------------
+
+def algorithmic_bytes(wl: W.Workload, slot_bytes: int) -> dict:
+    """Bytes one request-step must move: the packed state (codes, scales, fp16 units) read and
+    written, q/k/v read, alpha/beta read, o written, the slot index read."""
+    esz = 2 if wl.io_dtype == W.IO_BF16 else 4
+    H = wl.n_heads
+    state = 2 * slot_bytes
+    io = H * (2 * wl.d_k + wl.d_v) * esz + H * wl.alpha_width * 4 + H * 4 + H * wl.d_v * 4 + 4
+    return {"state": state, "io": io, "total": state + io}
+
+
+def peaks() -> tuple[float, str]:
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def source_digest() -> str:
+    h = hashlib.sha256()
+    for p in sorted(glob.glob(os.path.join(ROOT, "bit_recurrent_state_gated_b200", "csrc", "*"))):
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch of the decode kernel from the committed ncu summary, if it was
+    taken on the current kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", f"k_decode_{workload}.md")
+    if not os.path.exists(p):
+        return None
+    digest = source_digest()
+    with open(p) as f:
+        for line in f:
+            if line.startswith("bench-traffic:"):
+                parts = dict(kv.split("=") for kv in line.split(":", 1)[1].split())
+                if parts.get("source") == digest:
+                    return float(parts["bytes_per_launch"])
+    return None
+
+
+# ---- clocks ------------------------------------------------------------------------------------
+
+class ClockSampler:
+    """Polls the SM clock and the throttle reasons through NVML while the timed region runs."""
+
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4}
+
+    def __init__(self, device_index: int, period_s: float = 0.002):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._t = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = self._handle(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _handle(self, idx):
+        import torch
+        nv = self.nv
+        try:
+            bus = torch.cuda.get_device_properties(idx).pci_bus_id
+            return nv.nvmlDeviceGetHandleByPciBusId(bus.encode() if isinstance(bus, str) else bus)
+        except Exception:
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            phys = int(vis.split(",")[idx]) if vis and vis.split(",")[idx].isdigit() else idx
+            return nv.nvmlDeviceGetHandleByIndex(phys)
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for name, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+
+    def summary(self):
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# ---- CPU oracle (baseline and reference arm) ----------------------------------------------------
+
+def oracle_rate(wl: W.Workload, seconds: float, t0: int = 0):
+    """Request-steps/s of the CPU oracle on a bounded sample of the workload: the first few
+    requests of the batch (all heads), stepped repeatedly until `seconds` of CPU time."""
+    import oracle
+    threads = oracle.default_threads()
+    n_req = max(1, min(wl.batch, threads))
+    lay = oracle.Layout(wl.n_heads, wl.d_k, wl.d_v, wl.unit, wl.gate, wl.fit_iters)
+    pool = oracle.Pool(lay, wl.bits(), n_req)
+    si = np.arange(n_req, dtype=np.int32)
+    pool.quantize(si, wl.initial_state(wl.slot_idx()[:n_req]))
+    done, t_start, t = 0, time.perf_counter(), t0
+    while True:
+        x = wl.step_inputs(t)
+        xs = {k: np.ascontiguousarray(v[:n_req]) for k, v in x.items()}
+        ts = time.perf_counter()
+        pool.decode_step(si, xs["q"], xs["k"], xs["v"], xs["alpha"], xs["beta"], threads=threads)
+        done += n_req
+        t += 1
+        if time.perf_counter() - t_start >= seconds:
+            break
+        _ = ts
+    el = time.perf_counter() - t_start
+    return done / el, threads, f"{n_req} requests x {wl.n_heads} heads, {t - t0} steps"
+
+
+# ---- GPU arm -----------------------------------------------------------------------------------
+
+def run_ours(args, info):
+    import torch
+
+    from bit_recurrent_state_gated_b200 import sq
+
+    dev = info.local_rank
+    torch.cuda.set_device(dev)
+    base = W.WORKLOADS[args.workload]
+    wl = base.scaled(seed=base.seed + 1000 * info.rank)  # each rank: its own requests
+    lay = sq.Layout(wl.slots, wl.n_heads, wl.d_k, wl.d_v, wl.unit, wl.gate, wl.io_dtype,
+                    wl.fit_iters, wl.window, wl.n_outliers)
+    bits = wl.bits()
+    pool = sq.StatePool(lay, bits, wl.pivot_mask())
+    si_np = wl.slot_idx()
+    si = torch.from_numpy(si_np).cuda()
+    for c in range(0, wl.batch, 64):  # initial states, quantized on the GPU in chunks
+        S0 = torch.from_numpy(wl.initial_state(si_np[c:c + 64])).cuda()
+        pool.quantize(si[c:c + 64], S0)
+    n_sets = max(1, min(args.steps + args.warmup, 8))
+    sets_host, sets_dev = [], []
+    for t in range(n_sets):
+        x = wl.step_inputs(t)
+        if wl.io_dtype == W.IO_BF16:
+            qkv = [torch.from_numpy(x[n + "_bf16"]).view(torch.bfloat16) for n in "qkv"]
+        else:
+            qkv = [torch.from_numpy(x[n]) for n in "qkv"]
+        host = [a.pin_memory() for a in qkv + [torch.from_numpy(x["alpha"]),
+                                               torch.from_numpy(x["beta"])]]
+        sets_host.append(host)
+        sets_dev.append([a.cuda() for a in host])
+    out = torch.empty((wl.batch, wl.n_heads, wl.d_v), dtype=torch.float32, device="cuda")
+    out_host = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    st_handle = stream.cuda_stream
+
+    def step(t):
+        q, k, v, a, b = sets_dev[t % n_sets]
+        sq.sq_decode_step(pool.handle, si.data_ptr(), wl.batch, q.data_ptr(), k.data_ptr(),
+                          v.data_ptr(), a.data_ptr(), b.data_ptr(), out.data_ptr(), st_handle)
+
+    for t in range(args.warmup):
+        flush.zero_()
+        step(t)
+    torch.cuda.synchronize()
+    st, flag = pool.status()
+    if st != sq.SQ_OK:
+        raise RuntimeError(f"device flag {flag} after warm-up")
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev) as clocks:
+        for t in range(args.steps):
+            flush.zero_()  # every timed step starts with a cold L2
+            ev[t][0].record(stream)
+            step(args.warmup + t)
+            ev[t][1].record(stream)
+        torch.cuda.synchronize()
+    dist.barrier()
+    kernel_ms = [a.elapsed_time(b) for a, b in ev]
+    dev_ms = dist.max_over_ranks(sum(kernel_ms), device="cuda")
+
+    # end to end: pinned host inputs -> device, step, o -> pinned host, every step
+    ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    d_in = [torch.empty_like(a) for a in sets_dev[0]]
+    dist.barrier()
+    torch.cuda.synchronize()
+    for t in range(args.steps):
+        flush.zero_()
+        ev2[t][0].record(stream)
+        for dst, src in zip(d_in, sets_host[(args.warmup + t) % n_sets]):
+            dst.copy_(src, non_blocking=True)
+        q, k, v, a, b = d_in
+        sq.sq_decode_step(pool.handle, si.data_ptr(), wl.batch, q.data_ptr(), k.data_ptr(),
+                          v.data_ptr(), a.data_ptr(), b.data_ptr(), out.data_ptr(), st_handle)
+        out_host.copy_(out, non_blocking=True)
+        ev2[t][1].record(stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    e2e_ms = dist.max_over_ranks(sum(a.elapsed_time(b) for a, b in ev2), device="cuda")
+    st, flag = pool.status()
+    if st != sq.SQ_OK:
+        raise RuntimeError(f"device flag {flag} in the timed region")
+    h2d = sum(a.numel() * a.element_size() for a in sets_host[0])
+    d2h = out_host.numel() * out_host.element_size()
+
+    total_req_steps = wl.batch * args.steps * info.world
+    ab = algorithmic_bytes(wl, pool.slot_bytes)
+    mean_launch_s = statistics.mean(kernel_ms) / 1e3
+    achieved = ab["total"] * wl.batch / mean_launch_s / 1e9
+    peak, peak_kind = peaks()
+    traffic = profiled_traffic(args.workload)
+    res = {
+        "metric": METRIC,
+        "value": total_req_steps / (dev_ms / 1e3),
+        "unit": UNIT,
+        "n_gpus": info.world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": dev_ms / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic (seeded; no dataset)",
+        "config": {
+            "workload": f"{wl.name}: {wl.notes}",
+            "batch_per_gpu": wl.batch, "heads": wl.n_heads, "d_k": wl.d_k, "d_v": wl.d_v,
+            "slots_per_gpu": wl.slots, "gate": "scalar" if wl.gate == 0 else "diagonal",
+            "io": "bf16" if wl.io_dtype == W.IO_BF16 else "f32", "fit_iters": wl.fit_iters,
+            "state_bytes_per_request": pool.slot_bytes,
+            "algorithmic_bytes_per_request_step": ab["total"],
+            "l2": "flushed (256 MB write) before every timed step",
+            "parallelism": f"dp{info.world} (requests partitioned, no collective)",
+        },
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)"
+                     if peak_kind == "measured" else "fallback 6.65 TB/s",
+                     "kernel": "k_decode", "mean_launch_us": mean_launch_s * 1e6},
+        "e2e": {"value": total_req_steps / (e2e_ms / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps,
+        "clocks": clocks.summary(),
+    }
+    if info.world == 1 and info.rank == 0:
+        rate, cores, sample = oracle_rate(wl, args.cpu_seconds)
+        res["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
+                               "sample": sample}
+    pool.close()
+    return res
+
+
+def run_reference(args, info):
+    """The CPU oracle as the reference arm, on the same workload and metric."""
+    if info.rank != 0:
+        return None
+    wl = W.WORKLOADS[args.workload]
+    per_step = max(0.5, min(args.cpu_seconds, 150.0 / max(1, args.steps + args.warmup)))
+    for t in range(args.warmup):
+        oracle_rate(wl, per_step / 4, t0=t)
+    rates, cores, sample = [], 0, ""
+    t0 = time.perf_counter()
+    for t in range(args.steps):
+        r, cores, sample = oracle_rate(wl, per_step, t0=args.warmup + t)
+        rates.append(r)
+    el = time.perf_counter() - t0
+    value = statistics.mean(rates)
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": info.world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": el / max(args.steps, 1) * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64 update, f32 state",
+        "data": "synthetic (seeded; no dataset)",
+        "config": {"workload": f"{wl.name}: {wl.notes}", "batch_per_gpu": wl.batch,
+                   "heads": wl.n_heads, "d_k": wl.d_k, "d_v": wl.d_v},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"per step: {sample}"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    info = dist.rank_info()
+    if args.impl == "reference":
+        res = run_reference(args, info)
+    else:
+        dist.init("nccl")
+        try:
+            res = run_ours(args, info)
+        finally:
+            dist.finalize()
+    if res is not None and info.rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,75 @@
+// sq_internal.h -- structures shared by the host API and the kernels of libsq.
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace sq {
+
+constexpr int kThreads = 256;  // 8 warps; warp w owns key rows [16w, 16w+16)
+constexpr int kMaxD = 128;     // d_k, d_v <= 128, multiples of 16
+constexpr int kSlack = 16;     // bytes after a staged head block (6-bit unpack reads ahead)
+
+// Per head, shared by all slots (the widths are fixed offline).
+struct HeadDesc {
+  uint32_t off;         // byte offset of the head block within a slot
+  uint32_t bytes;       // block bytes, a multiple of 16
+  uint32_t pivot_head;  // 1: the head is one fp16 matrix (no scales)
+  uint32_t width;       // head units: the width; key-row units: 0 (see the row table)
+};
+
+// Row table: rows[h * d_k + i] = (byte offset of row i within the head block) << 8 | width,
+// width 16 for an fp16 pivot row.
+__host__ __device__ inline uint32_t row_off(uint32_t d) { return d >> 8; }
+__host__ __device__ inline int row_width(uint32_t d) { return (int)(d & 0xff); }
+
+struct StepArgs {
+  uint8_t* pool;
+  int64_t slot_bytes;
+  int32_t n_slots;
+  const int32_t* slot_idx;
+  int32_t batch;
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* alpha;
+  const float* beta;
+  float* out;
+  float* s_new;  // optional fp32 state after the update (tests)
+  const HeadDesc* heads;
+  const uint32_t* rows;
+  int32_t H, dk, dv, fit_iters;
+  uint32_t stage_bytes;  // smem bytes reserved for one staged head block
+  int32_t* flag;
+  // windowed variant
+  uint8_t* side;          // side region base (n_slots * side_slot_bytes)
+  int64_t side_slot_bytes;
+  int32_t window, n_outliers;
+};
+
+struct QuantArgs {
+  uint8_t* pool;
+  int64_t slot_bytes;
+  int32_t n_slots;
+  const int32_t* slot_idx;
+  int32_t n;
+  const float* S;  // quantize: input; dequantize: output (cast away const)
+  float* S_out;
+  const HeadDesc* heads;
+  const uint32_t* rows;
+  int32_t H, dk, dv, fit_iters, n_outliers;
+  uint32_t stage_bytes;
+  int32_t* flag;
+  uint8_t* side;
+  int64_t side_slot_bytes;
+};
+
+// Launchers (sq_kernels.cu). Return cudaSuccess or the launch error.
+cudaError_t launch_decode(const StepArgs& a, int gate, int io, bool want_state, int num_sms,
+                          cudaStream_t st);
+cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t st);
+cudaError_t launch_dequantize(const QuantArgs& a, cudaStream_t st);
+cudaError_t launch_window_step(const StepArgs& a, int gate, int io, int num_sms,
+                               cudaStream_t st);
+cudaError_t launch_window_flush(const StepArgs& a, int num_sms, cudaStream_t st);
+
+}  // namespace sq

@@ -1,0 +1,183 @@
+/*
+ * sq.h -- C ABI of libsq: the per-token decode step of gated delta-rule linear attention over
+ * a pool of per-request recurrent states held in a packed, mixed-width, dual-axis-scaled
+ * format, on NVIDIA B200 (sm_100a).
+ *
+ * Sources (prose web pages; no formulas or code are printed there):
+ *   [SQ-E] STEPQuant explainer (blog.ontle.kr/blog/302)
+ *   [SQ-N] STEPQuant news, "STEPQuant、推論メモリを最大68.7%削減", section 研究の概要
+ *   [LQ-N] LeapQuant news, "LeapQuant、線形注意の推論を1.47倍高速化", section 研究の概要
+ *
+ * Conventions for every call
+ *   - Pointers marked (device) are CUDA device pointers; (host) are ordinary host pointers.
+ *     Device pointers must be 16-byte aligned; the pool buffer must be 256-byte aligned.
+ *   - The caller owns every buffer it passes. The pool handle owns only its host metadata and
+ *     a few small device tables (offset tables and a status word), allocated at create and
+ *     freed at destroy.
+ *   - `stream` is a cudaStream_t passed as void*; NULL means the legacy default stream. Calls
+ *     that take a stream only enqueue work and return; they do not synchronize.
+ *   - Every call returns an sq_status. Nothing aborts, traps or prints. Argument errors are
+ *     found on the host before anything is enqueued. Problems only the GPU can see (a slot
+ *     index out of range, a non-finite input, a state too large for fp16 scales) set a sticky
+ *     device status word, and the affected (request, head) is skipped: its slot bytes stay as
+ *     they were and its output row is filled with NaN. sq_pool_status() reads and clears it.
+ *   - Within one call every slot index must be distinct; duplicates are not detected and give
+ *     an undefined result. Calls on one pool must not overlap in time on different streams.
+ *   - State layout: S[i][j] with i the key channel ("key row", [SQ-E] fitting paragraph) and
+ *     j the value channel ("value column", [SQ-N]). Dense fp32 states are row-major
+ *     [n][n_heads][d_k][d_v].
+ */
+#ifndef SQ_H
+#define SQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SQ_API __attribute__((visibility("default")))
+#else
+#define SQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SQ_OK = 0,
+  SQ_ERR_INVALID_ARG = 1, /* bad layout, bit map, pointer, alignment or size */
+  SQ_ERR_UNSUPPORTED = 2, /* a valid request this build does not handle (e.g. no sm_100 GPU) */
+  SQ_ERR_CUDA = 3,        /* a CUDA runtime call failed */
+  SQ_ERR_OOM = 4,         /* the pool's small device tables could not be allocated */
+  SQ_ERR_DEVICE_FLAG = 5, /* sq_pool_status: the GPU flagged a slot, a value or a range */
+  SQ_ERR_TIMEOUT = 6      /* sq_pool_status: a kernel gave up waiting on a copy */
+} sq_status;
+
+typedef enum { SQ_GATE_SCALAR = 0 /* GDN: one alpha per head */,
+               SQ_GATE_DIAG = 1 /* KDA: one alpha per key channel */ } sq_gate;
+typedef enum { SQ_UNIT_HEAD = 0 /* one width per head */,
+               SQ_UNIT_KEY_ROW = 1 /* one width per key row */ } sq_unit;
+typedef enum { SQ_IO_F32 = 0, SQ_IO_BF16 = 1 } sq_io_dtype; /* dtype of q, k, v */
+
+/* Bits of the device status word returned by sq_pool_status(). */
+#define SQ_FLAG_BAD_SLOT 1  /* a slot index outside [0, n_slots) */
+#define SQ_FLAG_NONFINITE 2 /* a non-finite q, k, v, alpha, beta or state value */
+#define SQ_FLAG_RANGE 4     /* a scale or fp16 value above the fp16 range */
+#define SQ_FLAG_TIMEOUT 8   /* a kernel stopped waiting for a bulk copy */
+
+/*
+ * Layout of one pool. [SQ-E] lifetime-aware allocation paragraph: a unit is a whole head
+ * (Qwen / GDN) or one key row (Kimi / KDA), and its width is fixed offline; the pool holds
+ * one state per concurrent request plus spare slots ([SQ-E], state-pool paragraph).
+ *   d_k, d_v     multiples of 16, at most 128.
+ *   fit_iters    alternations of the row/column max-abs scale fit, 1..8 (2 by default).
+ *   window       1: requantize after every token. W > 1: requantize after every W tokens,
+ *                holding the update at full precision in between ([LQ-N]).
+ *   n_outliers   per head, the entries of largest |S| kept in fp16 at each requantization
+ *                ([LQ-N], "compensation tokens"); 0..64, only with window > 1.
+ */
+typedef struct {
+  int32_t n_slots, n_heads, d_k, d_v;
+  int32_t unit;     /* sq_unit */
+  int32_t gate;     /* sq_gate */
+  int32_t io_dtype; /* sq_io_dtype */
+  int32_t fit_iters;
+  int32_t window;
+  int32_t n_outliers;
+} sq_layout;
+
+typedef struct sq_pool sq_pool;
+
+/*
+ * Packed format ([SQ-E] limitations paragraph: compressed values packed densely; efficiency
+ * paragraph: the compression ratio follows from the storage format).
+ *   bits_map (host): [n_heads] for SQ_UNIT_HEAD, [n_heads][d_k] for SQ_UNIT_KEY_ROW; values
+ *     2, 4, 6 or 8, or 16 for an FP16 pivot unit ([SQ-E]: a few high-risk units stay FP16).
+ *   pivot_mask (host, may be NULL): same shape; nonzero exactly where bits_map is 16.
+ * A quantized head block is r16[d_k] | c16[d_v] | rows | outliers: fp16 row and column
+ * scales, then row i as a little-endian bit stream in which element j holds the offset code
+ * code + 2^(b-1) (code in [-(2^(b-1)-1), 2^(b-1)-1]) at bits [j*b, (j+1)*b); a pivot row is
+ * the same stream of fp16 bit patterns. A pivot head (head units) is its fp16 matrix. Each
+ * head block is padded to 16 bytes; a slot is the heads in order. With window > 1 a side
+ * region follows the slots (per slot: the token count of the open window and the
+ * full-precision update held as low-rank factors).
+ *
+ * sq_pool_required_bytes: size in bytes of the device buffer a pool with this layout needs.
+ */
+SQ_API sq_status sq_pool_required_bytes(const sq_layout* layout, const uint8_t* bits_map,
+                                 const uint8_t* pivot_mask, size_t* bytes);
+
+/* Create a pool over a caller-owned device buffer (at least sq_pool_required_bytes, 256-byte
+ * aligned; contents are not touched until a quantize or step call). bits_map and pivot_mask
+ * are copied. On success *out receives the handle. Must be called with the buffer's device
+ * current. */
+SQ_API sq_status sq_state_pool_create(const sq_layout* layout, const uint8_t* bits_map,
+                               const uint8_t* pivot_mask, void* device_buf,
+                               size_t device_buf_bytes, sq_pool** out);
+
+/* Free the handle and its device tables (not the caller's buffer). NULL is accepted. */
+SQ_API sq_status sq_state_pool_destroy(sq_pool* pool);
+
+/* Geometry of a pool: bytes per slot, byte offset of each head block within a slot
+ * (head_offsets: host array of n_heads, may be NULL), and bytes per slot of the windowed side
+ * region (0 when window == 1; it starts at n_slots * slot_bytes). */
+SQ_API sq_status sq_pool_info(const sq_pool* pool, size_t* slot_bytes, size_t* head_offsets,
+                       size_t* side_bytes_per_slot);
+
+/* Quantize dense fp32 states into slots (cold start; [SQ-E] experimental setup uses the FP32
+ * state as baseline, so a pool is filled from fp32 states).
+ *   slot_idx (device) [n]; S (device) fp32 [n][n_heads][d_k][d_v].
+ * Fits the dual-axis scales, rounds pivots and outliers to fp16, packs, and (window > 1)
+ * closes the slot's window. */
+SQ_API sq_status sq_quantize_fp32_state(sq_pool* pool, const int32_t* slot_idx, int32_t n,
+                                 const float* S, void* stream);
+
+/* Dequantize slots to dense fp32: S_out[i][j] = fl32(code * r16_i * c16_j); pivots and
+ * outliers as their fp16 values. With window > 1 this is the frozen state (the open window's
+ * update is not included).
+ *   slot_idx (device) [n]; S_out (device) fp32 [n][n_heads][d_k][d_v]. */
+SQ_API sq_status sq_dequantize_state(sq_pool* pool, const int32_t* slot_idx, int32_t n,
+                              float* S_out, void* stream);
+
+/*
+ * One decode step for `batch` requests ([SQ-E] experimental-setup paragraph: the state is
+ * unpacked, updated and written back by one fused kernel at every decode step, and the two
+ * scales are refit on the updated state at every step; [SQ-E] paragraph introducing the gated
+ * Delta rule). For request b, head h, with M the state of slot slot_idx[b]:
+ *   S' = D M  (D = alpha I, or diag(alpha_i) for SQ_GATE_DIAG);  u = S'^T k;
+ *   b = beta (v - u);  M_new = S' + k b^T;  out = M_new^T q;
+ * then M_new's row and column scales are refit and it is requantized in place.
+ *   slot_idx (device) int32 [batch]
+ *   q, k (device) [batch][n_heads][d_k], v (device) [batch][n_heads][d_v], in io_dtype
+ *   alpha (device) fp32 [batch][n_heads] (scalar gate) or [batch][n_heads][d_k] (diagonal)
+ *   beta (device) fp32 [batch][n_heads]
+ *   out (device) fp32 [batch][n_heads][d_v]
+ * With window > 1 the frozen block is only read; the update goes to the side region, and the
+ * block is requantized after the W-th token of the window ([LQ-N]).
+ */
+SQ_API sq_status sq_decode_step(sq_pool* pool, const int32_t* slot_idx, int32_t batch, const void* q,
+                         const void* k, const void* v, const float* alpha, const float* beta,
+                         float* out, void* stream);
+
+/* Windowed pools: fold each listed slot's open window into its quantized block now and close
+ * the window (no-op for a closed window). slot_idx (device) [n]. */
+SQ_API sq_status sq_window_flush(sq_pool* pool, const int32_t* slot_idx, int32_t n, void* stream);
+
+/* Synchronize the device, read and clear the status word (*device_flag, may be NULL).
+ * Returns SQ_OK, SQ_ERR_DEVICE_FLAG or SQ_ERR_TIMEOUT. */
+SQ_API sq_status sq_pool_status(sq_pool* pool, int32_t* device_flag);
+
+/* Text of a status code (static storage). */
+SQ_API const char* sq_status_string(sq_status status);
+
+/* As sq_decode_step (window == 1 only), and also writes the fp32 state after the update and
+ * before requantization to s_new (device) fp32 [batch][n_heads][d_k][d_v]. For tests. */
+SQ_API sq_status sq_debug_decode_step_fp32(sq_pool* pool, const int32_t* slot_idx, int32_t batch,
+                                    const void* q, const void* k, const void* v,
+                                    const float* alpha, const float* beta, float* out,
+                                    float* s_new, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SQ_H */

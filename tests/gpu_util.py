@@ -1,0 +1,139 @@
+"""Helpers for the GPU parity tests: a libsq pool driven through the C ABI next to an oracle
+pool fed the same bytes and the same inputs."""
+from __future__ import annotations
+
+import numpy as np
+
+import oracle
+from bit_recurrent_state_gated_b200 import sq
+from bit_recurrent_state_gated_b200 import workloads as W
+
+import packed
+
+ATOL, RTOL = 2e-3, 1e-3  # |gpu - oracle| <= ATOL + RTOL |oracle|
+
+
+def sq_layout(wl, n_slots=None) -> sq.Layout:
+    return sq.Layout(n_slots or wl.slots, wl.n_heads, wl.d_k, wl.d_v, wl.unit, wl.gate,
+                     wl.io_dtype, wl.fit_iters, wl.window, wl.n_outliers)
+
+
+def orc_layout(wl) -> oracle.Layout:
+    return oracle.Layout(wl.n_heads, wl.d_k, wl.d_v, wl.unit, wl.gate, wl.fit_iters, wl.window,
+                         wl.n_outliers)
+
+
+def to_dev(a, dtype=None):
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(a))
+    if dtype is not None:
+        t = t.view(dtype)
+    return t.cuda()
+
+
+class GpuCase:
+    """A pool on the GPU for workload `wl`, filled from the workload's initial states."""
+
+    def __init__(self, wl: W.Workload, init=True):
+        import torch
+        self.wl = wl
+        self.bits = wl.bits()
+        self.pool = sq.StatePool(sq_layout(wl), self.bits, wl.pivot_mask())
+        self.si_np = wl.slot_idx()
+        self.si = to_dev(self.si_np)
+        if init:
+            S0 = to_dev(wl.initial_state(self.si_np))
+            self.pool.quantize(self.si, S0)
+            torch.cuda.synchronize()
+
+    def slots(self) -> np.ndarray:
+        import torch
+        torch.cuda.synchronize()
+        return self.pool.slots_view().cpu().numpy()
+
+    def device_inputs(self, x: dict):
+        import torch
+        if self.wl.io_dtype == W.IO_BF16:
+            q, k, v = (to_dev(x[n + "_bf16"], torch.bfloat16) for n in ("q", "k", "v"))
+        else:
+            q, k, v = (to_dev(x[n]) for n in ("q", "k", "v"))
+        return q, k, v, to_dev(x["alpha"]), to_dev(x["beta"])
+
+    def step(self, x: dict, want_state=False, slot_idx=None):
+        import torch
+        wl = self.wl
+        si = self.si if slot_idx is None else slot_idx
+        B = si.numel()
+        q, k, v, a, b = self.device_inputs(x)
+        out = torch.empty((B, wl.n_heads, wl.d_v), dtype=torch.float32, device="cuda")
+        s_new = (torch.empty((B, wl.n_heads, wl.d_k, wl.d_v), dtype=torch.float32,
+                             device="cuda") if want_state else None)
+        self.pool.decode_step(si, q, k, v, a, b, out, s_new)
+        torch.cuda.synchronize()
+        return out.cpu().numpy(), (s_new.cpu().numpy() if want_state else None)
+
+
+def oracle_pool_from(wl, bits, slot_bytes: np.ndarray) -> oracle.Pool:
+    """An oracle pool whose slots 0..n-1 hold the given packed slots."""
+    p = oracle.Pool(orc_layout(wl), bits, slot_bytes.shape[0])
+    assert p.slot_bytes == slot_bytes.shape[1]
+    p.data[:] = slot_bytes.reshape(-1)
+    return p
+
+
+def sub_inputs(x: dict, rows) -> dict:
+    return {k: np.ascontiguousarray(v[rows]) for k, v in x.items()}
+
+
+def close(got, ref, what: str):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    err = np.abs(got - ref)
+    bad = err > ATOL + RTOL * np.abs(ref)
+    assert not bad.any(), (f"{what}: {bad.sum()} of {bad.size} outside tolerance, "
+                           f"max err {err.max():.3g}")
+    return float(err.max())
+
+
+def compare_codes(wl, bits, gpu_slots: np.ndarray, orc_slots: np.ndarray, what: str):
+    """Codes equal on >= 99.99 % of quantized elements and within 1 LSB elsewhere; the
+    dequantized states within tolerance wherever codes match (fp16 entries always)."""
+    dg = packed.decode(gpu_slots, wl.unit, bits, wl.n_heads, wl.d_k, wl.d_v, wl.n_outliers)
+    do = packed.decode(orc_slots, wl.unit, bits, wl.n_heads, wl.d_k, wl.d_v, wl.n_outliers)
+    quant = ~np.broadcast_to(dg["pivot"][None, :, :, None], dg["codes"].shape)
+    if wl.n_outliers:
+        quant = quant & (dg["f16"] == 0) & (do["f16"] == 0)
+    diff = np.abs(dg["codes"] - do["codes"])[quant]
+    n_mis = int((diff != 0).sum())
+    frac = n_mis / max(diff.size, 1)
+    assert diff.size == 0 or diff.max() <= 1, f"{what}: code differs by {diff.max()} LSB"
+    assert frac <= 1e-4, f"{what}: {n_mis} of {diff.size} codes differ ({frac:.2e})"
+    Dg, Do = packed.dequant(dg), packed.dequant(do)
+    same = (dg["codes"] == do["codes"]) | ~quant
+    close(Dg[same], Do[same], what + " dequantized state")
+    return n_mis, diff.size
+
+
+def lockstep(case: GpuCase, t: int, sample=None, want_state=True):
+    """One GPU step checked against the oracle started from the GPU's own pre-step bytes.
+    `sample`: request indices to check (default all)."""
+    wl = case.wl
+    x = wl.step_inputs(t)
+    pre = case.slots()
+    o_gpu, s_gpu = case.step(x, want_state=want_state)
+    post = case.slots()
+    rows = np.arange(wl.batch) if sample is None else np.asarray(sample)
+    slots = case.si_np[rows]
+    opool = oracle_pool_from(wl, case.bits, pre[slots])
+    xs = sub_inputs(x, rows)
+    o_ref, s_ref = opool.decode_step(np.arange(rows.size), xs["q"], xs["k"], xs["v"],
+                                     xs["alpha"], xs["beta"], want_state=True)
+    close(o_gpu[rows], o_ref, f"step {t} o")
+    if want_state:
+        close(s_gpu[rows], s_ref, f"step {t} state after update")
+    n_mis, n = compare_codes(wl, case.bits, post[slots], opool.data.reshape(rows.size, -1),
+                             f"step {t}")
+    untouched = np.setdiff1d(np.arange(wl.slots), case.si_np)
+    if untouched.size:
+        np.testing.assert_array_equal(post[untouched], pre[untouched])
+    return n_mis, n
