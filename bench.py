@@ -101,8 +101,10 @@ def profiled_traffic(workload: str):
 class ClockSampler:
     """Polls the SM clock and the throttle reasons through NVML while the timed region runs."""
 
-    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
-               "sw_power_cap": 0x4}
+    REASONS = {"hw_slowdown": "nvmlClocksEventReasonHwSlowdown",
+               "sw_thermal_slowdown": "nvmlClocksEventReasonSwThermalSlowdown",
+               "hw_thermal_slowdown": "nvmlClocksEventReasonHwThermalSlowdown",
+               "sw_power_cap": "nvmlClocksEventReasonSwPowerCap"}
 
     def __init__(self, device_index: int, period_s: float = 0.002):
         self.samples, self.reasons, self.max_mhz = [], set(), None
@@ -122,8 +124,10 @@ class ClockSampler:
         import torch
         nv = self.nv
         try:
-            bus = torch.cuda.get_device_properties(idx).pci_bus_id
-            return nv.nvmlDeviceGetHandleByPciBusId(bus.encode() if isinstance(bus, str) else bus)
+            p = torch.cuda.get_device_properties(idx)
+            bus = "%08X:%02X:%02X.0" % (int(p.pci_domain_id), int(p.pci_bus_id),
+                                         int(p.pci_device_id))
+            return nv.nvmlDeviceGetHandleByPciBusId(bus.encode())
         except Exception:
             vis = os.environ.get("CUDA_VISIBLE_DEVICES")
             phys = int(vis.split(",")[idx]) if vis and vis.split(",")[idx].isdigit() else idx
@@ -135,8 +139,8 @@ class ClockSampler:
             try:
                 self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
                 r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-                for name, bit in self.REASONS.items():
-                    if r & bit:
+                for name, const in self.REASONS.items():
+                    if r & int(getattr(nv, const, 0)):
                         self.reasons.add(name)
             except Exception:
                 pass
@@ -171,19 +175,19 @@ def oracle_rate(wl: W.Workload, seconds: float, t0: int = 0):
     pool = oracle.Pool(lay, wl.bits(), n_req)
     si = np.arange(n_req, dtype=np.int32)
     pool.quantize(si, wl.initial_state(wl.slot_idx()[:n_req]))
-    done, t_start, t = 0, time.perf_counter(), t0
-    while True:
+    sets = []
+    for t in range(t0, t0 + 4):
         x = wl.step_inputs(t)
-        xs = {k: np.ascontiguousarray(v[:n_req]) for k, v in x.items()}
+        sets.append({k: np.ascontiguousarray(v[:n_req]) for k, v in x.items()})
+    done, busy, n = 0, 0.0, 0
+    while busy < seconds:  # only the oracle's own calls are timed
+        xs = sets[n % len(sets)]
         ts = time.perf_counter()
         pool.decode_step(si, xs["q"], xs["k"], xs["v"], xs["alpha"], xs["beta"], threads=threads)
+        busy += time.perf_counter() - ts
         done += n_req
-        t += 1
-        if time.perf_counter() - t_start >= seconds:
-            break
-        _ = ts
-    el = time.perf_counter() - t_start
-    return done / el, threads, f"{n_req} requests x {wl.n_heads} heads, {t - t0} steps"
+        n += 1
+    return done / busy, threads, f"{n_req} requests x {wl.n_heads} heads, {n} steps"
 
 
 # ---- GPU arm -----------------------------------------------------------------------------------
@@ -220,7 +224,16 @@ def run_ours(args, info):
         sets_dev.append([a.cuda() for a in host])
     out = torch.empty((wl.batch, wl.n_heads, wl.d_v), dtype=torch.float32, device="cuda")
     out_host = torch.empty(out.shape, dtype=torch.float32).pin_memory()
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    flush_buf = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    sink = torch.empty(1, dtype=torch.float32, device="cuda")
+
+    class _Flush:  # write then read a buffer twice the size of L2: L2 holds only clean lines
+        @staticmethod
+        def zero_():
+            flush_buf.zero_()
+            torch.sum(flush_buf, dim=0, keepdim=True, out=sink)
+
+    flush = _Flush()
     stream = torch.cuda.current_stream()
     st_handle = stream.cuda_stream
 
@@ -229,6 +242,7 @@ def run_ours(args, info):
         sq.sq_decode_step(pool.handle, si.data_ptr(), wl.batch, q.data_ptr(), k.data_ptr(),
                           v.data_ptr(), a.data_ptr(), b.data_ptr(), out.data_ptr(), st_handle)
 
+    log(f"pool ready: {wl.slots} slots x {pool.slot_bytes} B; warm-up")
     for t in range(args.warmup):
         flush.zero_()
         step(t)
@@ -249,6 +263,7 @@ def run_ours(args, info):
             ev[t][1].record(stream)
         torch.cuda.synchronize()
     dist.barrier()
+    log("timed region done")
     kernel_ms = [a.elapsed_time(b) for a, b in ev]
     dev_ms = dist.max_over_ranks(sum(kernel_ms), device="cuda")
 
@@ -303,7 +318,7 @@ def run_ours(args, info):
             "io": "bf16" if wl.io_dtype == W.IO_BF16 else "f32", "fit_iters": wl.fit_iters,
             "state_bytes_per_request": pool.slot_bytes,
             "algorithmic_bytes_per_request_step": ab["total"],
-            "l2": "flushed (256 MB write) before every timed step",
+            "l2": "flushed before every timed step (write, then read, 256 MB)",
             "parallelism": f"dp{info.world} (requests partitioned, no collective)",
         },
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
@@ -316,8 +331,10 @@ def run_ours(args, info):
         "gpu_launches": args.steps,
         "clocks": clocks.summary(),
     }
+    log("end-to-end region done")
     if info.world == 1 and info.rank == 0:
         rate, cores, sample = oracle_rate(wl, args.cpu_seconds)
+        log("cpu baseline done")
         res["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
                                "sample": sample}
     pool.close()
@@ -353,7 +370,14 @@ def run_reference(args, info):
     }
 
 
+def log(msg: str):
+    sys.stderr.write(f"[bench {time.strftime('%H:%M:%S')}] {msg}\n")
+    sys.stderr.flush()
+
+
 def main():
+    import faulthandler
+    faulthandler.enable()
     args = parse()
     info = dist.rank_info()
     if args.impl == "reference":

@@ -3,10 +3,11 @@
 // never aborts or prints.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <new>
 #include <vector>
 
-#include "../../include/sq.h"
+#include "sq.h"
 #include "sq_internal.h"
 
 struct sq_pool {
@@ -17,8 +18,10 @@ struct sq_pool {
   size_t slot_bytes = 0, side_slot_bytes = 0, side_head_bytes = 0;
   uint32_t max_head_bytes = 0;
   uint8_t* base = nullptr;  // caller's buffer
+  std::vector<int32_t> order;  // heads sorted by width (pivot heads last)
   sq::HeadDesc* d_heads = nullptr;
   uint32_t* d_rows = nullptr;
+  int32_t* d_order = nullptr;
   int32_t* d_flag = nullptr;
   int device = 0, num_sms = 0;
 };
@@ -86,6 +89,12 @@ sq_status plan(const sq_layout* L, const uint8_t* bits, const uint8_t* pivot_mas
   }
   P->slot_bytes = off;
   P->max_head_bytes = maxb;
+  P->order.resize(H);
+  for (int h = 0; h < H; ++h) P->order[h] = h;
+  std::stable_sort(P->order.begin(), P->order.end(), [&](int x, int y) {
+    const auto key = [&](int h) { return P->heads[h].pivot_head ? 99 : (int)P->heads[h].width; };
+    return key(x) < key(y);
+  });
   if (L->window > 1) {
     // per slot: 16-byte header (token count) then, per head, the cumulative gate g (d_k
     // floats) and `window` low-rank terms (k_hat [d_k], b [d_v] fp32)
@@ -127,10 +136,12 @@ sq::StepArgs step_args(sq_pool* p, const int32_t* slot_idx, int32_t batch, const
   a.s_new = s_new;
   a.heads = p->d_heads;
   a.rows = p->d_rows;
+  a.order = p->d_order;
   a.H = p->L.n_heads;
   a.dk = p->L.d_k;
   a.dv = p->L.d_v;
   a.fit_iters = p->L.fit_iters;
+  a.per_row = p->L.unit == SQ_UNIT_KEY_ROW;
   a.stage_bytes = p->max_head_bytes;
   a.flag = p->d_flag;
   a.side = p->side_slot_bytes ? p->base + (size_t)p->L.n_slots * p->slot_bytes : nullptr;
@@ -216,6 +227,10 @@ sq_status sq_state_pool_create(const sq_layout* layout, const uint8_t* bits_map,
   if (e == cudaSuccess) e = cudaMalloc(&p->d_heads, sizeof(sq::HeadDesc) * p->heads.size());
   if (e == cudaSuccess) e = cudaMalloc(&p->d_rows, sizeof(uint32_t) * p->rows.size());
   if (e == cudaSuccess) e = cudaMalloc(&p->d_flag, sizeof(int32_t));
+  if (e == cudaSuccess) e = cudaMalloc(&p->d_order, sizeof(int32_t) * p->order.size());
+  if (e == cudaSuccess)
+    e = cudaMemcpy(p->d_order, p->order.data(), sizeof(int32_t) * p->order.size(),
+                   cudaMemcpyHostToDevice);
   if (e == cudaSuccess)
     e = cudaMemcpy(p->d_heads, p->heads.data(), sizeof(sq::HeadDesc) * p->heads.size(),
                    cudaMemcpyHostToDevice);
@@ -227,6 +242,7 @@ sq_status sq_state_pool_create(const sq_layout* layout, const uint8_t* bits_map,
     cudaFree(p->d_heads);
     cudaFree(p->d_rows);
     cudaFree(p->d_flag);
+    cudaFree(p->d_order);
     delete p;
     return cuda_status(e);
   }
@@ -239,6 +255,7 @@ sq_status sq_state_pool_destroy(sq_pool* pool) {
   cudaFree(pool->d_heads);
   cudaFree(pool->d_rows);
   cudaFree(pool->d_flag);
+  cudaFree(pool->d_order);
   delete pool;
   return SQ_OK;
 }

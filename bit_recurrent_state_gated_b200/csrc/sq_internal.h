@@ -9,6 +9,10 @@ constexpr int kThreads = 256;  // 8 warps; warp w owns key rows [16w, 16w+16)
 constexpr int kMaxD = 128;     // d_k, d_v <= 128, multiples of 16
 constexpr int kSlack = 16;     // bytes after a staged head block (6-bit unpack reads ahead)
 
+// Device status word bits (the same values as SQ_FLAG_* in include/sq.h).
+constexpr int32_t SQ_FLAG_BAD_SLOT_BIT = 1, SQ_FLAG_NONFINITE_BIT = 2, SQ_FLAG_RANGE_BIT = 4,
+                  SQ_FLAG_TIMEOUT_BIT = 8;
+
 // Per head, shared by all slots (the widths are fixed offline).
 struct HeadDesc {
   uint32_t off;         // byte offset of the head block within a slot
@@ -37,7 +41,9 @@ struct StepArgs {
   float* s_new;  // optional fp32 state after the update (tests)
   const HeadDesc* heads;
   const uint32_t* rows;
+  const int32_t* order;  // heads sorted by width: items run head-major in this order
   int32_t H, dk, dv, fit_iters;
+  int32_t per_row;       // 1: key-row units (the row table is staged with each head block)
   uint32_t stage_bytes;  // smem bytes reserved for one staged head block
   int32_t* flag;
   // windowed variant

@@ -1,0 +1,330 @@
+// sq_tile.cuh -- shared device code of libsq's kernels (sm_100a): the tile mapping, the
+// alternating dual-axis fit, requantize + pack, and the top-n compensation entries.
+//
+// One CTA of 256 threads handles one (request, head) state tile at a time: warp w owns key
+// rows [16w, 16w+16), lane l owns value columns [4l, 4l+4), so every thread keeps 16 x 4 fp32
+// state values in registers and each packed row is read and written by one warp (a row's
+// width is warp-uniform even when widths vary per key row).
+#pragma once
+#include <cuda_runtime.h>
+#include <math.h>
+
+#include <type_traits>
+
+#include "sq_device.cuh"
+#include "sq_internal.h"
+
+namespace sq {
+namespace tile {
+
+constexpr int kWarps = kThreads / 32;
+constexpr int kRows = 16;  // rows per warp
+enum { MODE_ROWS = 0, MODE_W2 = 2, MODE_W4 = 4, MODE_W6 = 6, MODE_W8 = 8, MODE_PIVOT = 16 };
+template <int M>
+using ModeT = std::integral_constant<int, M>;
+
+__host__ __device__ constexpr uint32_t round16(uint32_t x) { return (x + 15u) & ~15u; }
+
+// Column arrays in shared memory (kMaxD floats each).
+enum { COL_C = 0, COL_IC, COL_B, COL_P, COL_X, COL_INV, COL_IC16, COL_V, N_COL };
+
+__device__ __forceinline__ float ld_io(const void* base, int io, int idx) {
+  if (io == 1) {
+    const uint16_t h = reinterpret_cast<const uint16_t*>(base)[idx];
+    return __uint_as_float(static_cast<uint32_t>(h) << 16);
+  }
+  return reinterpret_cast<const float*>(base)[idx];
+}
+
+__device__ __forceinline__ int q_of_width(int b) { return b == 16 ? 0 : (1 << (b - 1)) - 1; }
+
+// Row and column scales of the tile held in S by alternating max-abs passes, the same rule as
+// the oracle: cold start c = 1; r_i = max(max_j fl(|S_ij| fl(1/c_j)) / Q_i, 2^-14);
+// w_i = fl(1 / fl(r_i Q_i)); c_j = max(max_i fl(|S_ij| w_i), 2^-14). Rows with Q = 0 (fp16
+// pivot rows) get w = 0 and drop out of the column maxima; zeroed elements (outliers, idle
+// lanes) contribute nothing. On return rowR[i] = r_i and col[COL_X][j] = c_j.
+__device__ __forceinline__ void fit_scales(const float (&S)[kRows][4], int fit_iters, int warp,
+                                           int lane, int dk, int dv, const uint32_t* rows,
+                                           float* rowW, float* rowR, float* rowtmp, float* red,
+                                           float* col) {
+  float inv_c[4] = {1.f, 1.f, 1.f, 1.f};
+  float* tmp = rowtmp + warp * kRows;
+  for (int it = 0; it < fit_iters; ++it) {
+    float rm[kRows];
+#pragma unroll
+    for (int s = 0; s < kRows; ++s) {
+      float m;
+      if (it == 0)
+        m = fmaxf(fmaxf(fabsf(S[s][0]), fabsf(S[s][1])), fmaxf(fabsf(S[s][2]), fabsf(S[s][3])));
+      else
+        m = fmaxf(fmaxf(fabsf(S[s][0]) * inv_c[0], fabsf(S[s][1]) * inv_c[1]),
+                  fmaxf(fabsf(S[s][2]) * inv_c[2], fabsf(S[s][3]) * inv_c[3]));
+      rm[s] = warp_max_nonneg(m);
+    }
+    if (lane == 0) {
+#pragma unroll
+      for (int s = 0; s < kRows; s += 4)
+        *reinterpret_cast<float4*>(tmp + s) = make_float4(rm[s], rm[s + 1], rm[s + 2], rm[s + 3]);
+    }
+    __syncwarp();
+    if (lane < kRows) {
+      const int i = warp * kRows + lane;
+      if (i < dk) {
+        const int Q = q_of_width(row_width(rows[i]));
+        float r = 0.f, w = 0.f;
+        if (Q > 0) {
+          r = fmaxf(__fdiv_rn(tmp[lane], (float)Q), kScaleFloor);
+          w = __frcp_rn(__fmul_rn(r, (float)Q));
+        }
+        rowR[i] = r;
+        rowW[i] = w;
+      } else {
+        rowW[i] = 0.f;
+      }
+    }
+    __syncwarp();
+    float cm[4] = {0.f, 0.f, 0.f, 0.f};
+    const float* wrow = rowW + warp * kRows;
+#pragma unroll
+    for (int s = 0; s < kRows; s += 4) {
+      const float4 w4 = *reinterpret_cast<const float4*>(wrow + s);
+      const float ws[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+      for (int t = 0; t < 4; ++t)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) cm[e] = fmaxf(cm[e], fabsf(S[s + t][e]) * ws[t]);
+    }
+    *reinterpret_cast<float4*>(red + warp * 2 * kMaxD + 4 * lane) =
+        make_float4(cm[0], cm[1], cm[2], cm[3]);
+    __syncthreads();
+    const int t = threadIdx.x;
+    if (t < dv) {
+      float c = 0.f;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) c = fmaxf(c, red[w * 2 * kMaxD + t]);
+      c = fmaxf(c, kScaleFloor);
+      col[COL_X * kMaxD + t] = c;
+      col[COL_INV * kMaxD + t] = __frcp_rn(c);
+    } else if (t < kMaxD) {  // columns past d_v: neutral values for the idle lanes
+      col[COL_X * kMaxD + t] = kScaleFloor;
+      col[COL_INV * kMaxD + t] = 1.f;
+    }
+    __syncthreads();
+    if (it + 1 < fit_iters) {
+      const float4 iv = *reinterpret_cast<const float4*>(col + COL_INV * kMaxD + 4 * lane);
+      inv_c[0] = iv.x;
+      inv_c[1] = iv.y;
+      inv_c[2] = iv.z;
+      inv_c[3] = iv.w;
+    }
+  }
+}
+
+// Round the fitted scales to fp16, check the fp16 range, quantize the tile and store scales
+// and packed rows to the head block `dst` (global memory). Codes: nearest-even integer to
+// fl(S_ij fl(1/r16_i)) * fl(1/c16_j) (the last product exact, inside one fma), clamped to
+// [-Q, Q]. Returns false (and stores nothing) if a scale or a pivot value overflows fp16.
+// Contains __syncthreads; *bad must be 0 on entry.
+template <int MODE>
+__device__ __forceinline__ bool requant_store(const float (&S)[kRows][4], uint8_t* dst,
+                                              const uint32_t* rows, int warp, int lane, int dk,
+                                              int dv, const float* rowR, float* rowIR,
+                                              float* col, int* bad) {
+  const bool active = 4 * lane < dv;
+  const int t = threadIdx.x;
+  if (lane < kRows) {
+    const int i = warp * kRows + lane;
+    if (i < dk) {
+      float ir = 0.f;
+      if (q_of_width(row_width(rows[i])) > 0) {
+        const __half r16 = __float2half_rn(rowR[i]);
+        if (__hisinf(r16)) atomicOr(bad, 1);
+        ir = __frcp_rn(__half2float(r16));
+      }
+      rowIR[i] = ir;
+    }
+  }
+  if (t < dv) {
+    const __half c16 = __float2half_rn(col[COL_X * kMaxD + t]);
+    if (__hisinf(c16)) atomicOr(bad, 1);
+    col[COL_IC16 * kMaxD + t] = __frcp_rn(__half2float(c16));
+  } else if (t < kMaxD) {
+    col[COL_IC16 * kMaxD + t] = 0.f;
+  }
+#pragma unroll
+  for (int s = 0; s < kRows; ++s) {
+    const int i = warp * kRows + s;
+    if (i < dk && row_width(rows[i]) == 16 && active && f16_overflows(S[s])) atomicOr(bad, 1);
+  }
+  __syncthreads();
+  if (*bad) return false;
+  if (lane < kRows) {
+    const int i = warp * kRows + lane;
+    if (i < dk)
+      reinterpret_cast<__half*>(dst)[i] = q_of_width(row_width(rows[i])) > 0
+                                             ? __float2half_rn(rowR[i])
+                                             : __float2half_rn(0.f);
+  }
+  if (t < dv) reinterpret_cast<__half*>(dst)[dk + t] = __float2half_rn(col[COL_X * kMaxD + t]);
+  const float4 ic4 = *reinterpret_cast<const float4*>(col + COL_IC16 * kMaxD + 4 * lane);
+  const float ic[4] = {ic4.x, ic4.y, ic4.z, ic4.w};
+#pragma unroll
+  for (int s = 0; s < kRows; ++s) {
+    const int i = warp * kRows + s;
+    if (i < dk) {
+      const uint32_t d = rows[i];
+      uint8_t* row = dst + row_off(d);
+      const int b = MODE == MODE_ROWS ? row_width(d) : MODE;
+      if (b == 16) {
+        store4_f16(row, lane, S[s], active);
+      } else {
+        const float ir = rowIR[i];
+        const float Q = (float)q_of_width(b);
+        const float magic = kMagic + (float)(1 << (b - 1));
+        float y[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float v = __fmaf_rn(__fmul_rn(S[s][e], ir), ic[e], magic);
+          y[e] = fminf(fmaxf(v, magic - Q), magic + Q);
+        }
+        switch (b) {
+          case 2: store4<2>(row, lane, y, active); break;
+          case 4: store4<4>(row, lane, y, active); break;
+          case 6: store4<6>(row, lane, y, active); break;
+          default: store4<8>(row, lane, y, active); break;
+        }
+      }
+    }
+  }
+  return true;
+}
+
+__device__ __forceinline__ bool requant_store_any(int mode, const float (&S)[kRows][4],
+                                                  uint8_t* dst, const uint32_t* rows, int warp,
+                                                  int lane, int dk, int dv, const float* rowR,
+                                                  float* rowIR, float* col, int* bad) {
+  switch (mode) {
+    case MODE_W2: return requant_store<MODE_W2>(S, dst, rows, warp, lane, dk, dv, rowR, rowIR, col, bad);
+    case MODE_W4: return requant_store<MODE_W4>(S, dst, rows, warp, lane, dk, dv, rowR, rowIR, col, bad);
+    case MODE_W6: return requant_store<MODE_W6>(S, dst, rows, warp, lane, dk, dv, rowR, rowIR, col, bad);
+    case MODE_W8: return requant_store<MODE_W8>(S, dst, rows, warp, lane, dk, dv, rowR, rowIR, col, bad);
+    default: return requant_store<MODE_ROWS>(S, dst, rows, warp, lane, dk, dv, rowR, rowIR, col, bad);
+  }
+}
+
+// fp16 pivot head: all 4 values per row rounded to fp16 and stored row-major. Contains
+// __syncthreads; false (nothing stored) if a value overflows fp16.
+__device__ __forceinline__ bool store_pivot_head(const float (&S)[kRows][4], uint8_t* dst,
+                                                 int warp, int lane, int dk, int dv, int* bad) {
+  const bool active = 4 * lane < dv;
+  bool of = false;
+#pragma unroll
+  for (int s = 0; s < kRows; ++s)
+    if (warp * kRows + s < dk && active) of |= f16_overflows(S[s]);
+  if (of) atomicOr(bad, 1);
+  __syncthreads();
+  if (*bad) return false;
+#pragma unroll
+  for (int s = 0; s < kRows; ++s) {
+    const int i = warp * kRows + s;
+    if (i < dk) store4_f16(dst + (size_t)i * 2 * dv, lane, S[s], active);
+  }
+  return true;
+}
+
+// Unpack the warp's rows of a staged head block into S (exact codes, or fp16 values for pivot
+// rows), zero outside the tile.
+template <int MODE>
+__device__ __forceinline__ void unpack_tile(float (&S)[kRows][4], const uint8_t* blk,
+                                            const uint32_t* rows, int warp, int lane, int dk,
+                                            int dv) {
+#pragma unroll
+  for (int s = 0; s < kRows; ++s) {
+    const int i = warp * kRows + s;
+    if (i < dk && 4 * lane < dv) {
+      const uint32_t d = rows[i];
+      const uint8_t* row = blk + row_off(d);
+      if constexpr (MODE == MODE_ROWS)
+        unpack4_rt(row_width(d), row, lane, S[s]);
+      else
+        unpack4<MODE>(row, lane, S[s]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) S[s][e] = 0.f;
+    }
+  }
+}
+
+__device__ __forceinline__ void unpack_tile_any(int mode, float (&S)[kRows][4],
+                                                const uint8_t* blk, const uint32_t* rows,
+                                                int warp, int lane, int dk, int dv) {
+  switch (mode) {
+    case MODE_W2: unpack_tile<MODE_W2>(S, blk, rows, warp, lane, dk, dv); break;
+    case MODE_W4: unpack_tile<MODE_W4>(S, blk, rows, warp, lane, dk, dv); break;
+    case MODE_W6: unpack_tile<MODE_W6>(S, blk, rows, warp, lane, dk, dv); break;
+    case MODE_W8: unpack_tile<MODE_W8>(S, blk, rows, warp, lane, dk, dv); break;
+    case MODE_PIVOT: unpack_tile<MODE_PIVOT>(S, blk, rows, warp, lane, dk, dv); break;
+    default: unpack_tile<MODE_ROWS>(S, blk, rows, warp, lane, dk, dv); break;
+  }
+}
+
+__device__ __forceinline__ int mode_of(const HeadDesc& hd) {
+  return hd.pivot_head ? MODE_PIVOT : (int)hd.width;  // width 0 = per-row widths
+}
+
+// ---------------------------------------------------------------------------------------------
+// Top-n entries of |S| over the quantized rows (ties to the lower flat index i*dv + j), by n
+// rounds of a CTA-wide arg-max. Selected elements are recorded in `sel` (bit s*4+e per thread)
+// and their (index, value) pairs in out_idx / out_val (smem, n entries, in selection order).
+// ---------------------------------------------------------------------------------------------
+__device__ __forceinline__ void select_top(const float (&S)[kRows][4], int n, int warp, int lane,
+                                           int dk, int dv, const uint32_t* rows, uint64_t& sel,
+                                           unsigned long long* wbest, int* out_idx,
+                                           float* out_val) {
+  sel = 0;
+  for (int r = 0; r < n; ++r) {
+    unsigned long long best = 0;
+#pragma unroll
+    for (int s = 0; s < kRows; ++s) {
+      const int i = warp * kRows + s;
+      if (i < dk && 4 * lane < dv && row_width(rows[i]) != 16) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if ((sel >> (s * 4 + e)) & 1) continue;
+          const uint32_t idx = (uint32_t)(i * dv + 4 * lane + e);
+          const unsigned long long key =
+              ((unsigned long long)__float_as_uint(fabsf(S[s][e])) << 32) | (0xffffffffu - idx);
+          best = key > best ? key : best;
+        }
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const unsigned long long other = __shfl_xor_sync(0xffffffffu, best, o);
+      best = other > best ? other : best;
+    }
+    if (lane == 0) wbest[warp] = best;
+    __syncthreads();
+    unsigned long long win = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) win = wbest[w] > win ? wbest[w] : win;
+    const uint32_t idx = 0xffffffffu - (uint32_t)(win & 0xffffffffu);
+    const int wi = (int)(idx / dv), wj = (int)(idx % dv);
+    if (win != 0 && wi / kRows == warp && wj / 4 == lane) {
+      const int s = wi % kRows, e = wj % 4;
+      sel |= 1ull << (s * 4 + e);
+      out_idx[r] = (int)idx;
+      float v = 0.f;
+#pragma unroll
+      for (int s2 = 0; s2 < kRows; ++s2)
+#pragma unroll
+        for (int e2 = 0; e2 < 4; ++e2)
+          if (s2 == s && e2 == e) v = S[s2][e2];
+      out_val[r] = v;
+    }
+    __syncthreads();
+  }
+}
+
+}  // namespace tile
+}  // namespace sq
