@@ -96,10 +96,12 @@ sq_status plan(const sq_layout* L, const uint8_t* bits, const uint8_t* pivot_mas
     return key(x) < key(y);
   });
   if (L->window > 1) {
-    // per slot: 16-byte header (token count) then, per head, the cumulative gate g (d_k
-    // floats) and `window` low-rank terms (k_hat [d_k], b [d_v] fp32)
-    P->side_head_bytes = 4u * (size_t)dk + (size_t)L->window * 4u * (size_t)(dk + dv);
-    P->side_slot_bytes = 16 + (size_t)H * P->side_head_bytes;
+    if (L->window > 64) return SQ_ERR_INVALID_ARG;
+    // per (slot, head): token count (16-byte header), the cumulative gate g (d_k fp32) and
+    // `window` low-rank terms (k_hat [d_k], b [d_v] fp32)
+    P->side_head_bytes = 16 + 4u * (size_t)dk + (size_t)L->window * 4u * (size_t)(dk + dv);
+    P->side_head_bytes = (P->side_head_bytes + 15) / 16 * 16;
+    P->side_slot_bytes = (size_t)H * P->side_head_bytes;
     P->side_slot_bytes = (P->side_slot_bytes + 255) / 256 * 256;
   }
   return SQ_OK;
@@ -146,6 +148,7 @@ sq::StepArgs step_args(sq_pool* p, const int32_t* slot_idx, int32_t batch, const
   a.flag = p->d_flag;
   a.side = p->side_slot_bytes ? p->base + (size_t)p->L.n_slots * p->slot_bytes : nullptr;
   a.side_slot_bytes = (int64_t)p->side_slot_bytes;
+  a.side_head_bytes = (int64_t)p->side_head_bytes;
   a.window = p->L.window;
   a.n_outliers = p->L.n_outliers;
   return a;
@@ -172,6 +175,7 @@ sq::QuantArgs quant_args(sq_pool* p, const int32_t* slot_idx, int32_t n, const f
   a.flag = p->d_flag;
   a.side = p->side_slot_bytes ? p->base + (size_t)p->L.n_slots * p->slot_bytes : nullptr;
   a.side_slot_bytes = (int64_t)p->side_slot_bytes;
+  a.side_head_bytes = (int64_t)p->side_head_bytes;
   return a;
 }
 

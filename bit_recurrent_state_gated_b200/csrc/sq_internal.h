@@ -48,7 +48,7 @@ struct StepArgs {
   int32_t* flag;
   // windowed variant
   uint8_t* side;          // side region base (n_slots * side_slot_bytes)
-  int64_t side_slot_bytes;
+  int64_t side_slot_bytes, side_head_bytes;
   int32_t window, n_outliers;
 };
 
@@ -66,7 +66,7 @@ struct QuantArgs {
   uint32_t stage_bytes;
   int32_t* flag;
   uint8_t* side;
-  int64_t side_slot_bytes;
+  int64_t side_slot_bytes, side_head_bytes;
 };
 
 // Launchers (sq_kernels.cu). Return cudaSuccess or the launch error.

@@ -10,26 +10,14 @@ using namespace tile;
 // ---------------------------------------------------------------------------------------------
 // Quantize dense fp32 states into slots: one CTA per (slot, head).
 // ---------------------------------------------------------------------------------------------
-constexpr int kMaxOutliers = 64;
-
-struct QSmem {
-  float red[kWarps * 2 * kMaxD];
-  float rowW[kMaxD], rowR[kMaxD], rowIR[kMaxD], rowtmp[kWarps * kRows];
-  float col[N_COL * kMaxD];
-  unsigned long long wbest[kWarps];
-  int oidx[kMaxOutliers];
-  float oval[kMaxOutliers];
-  int misc[4];
-};
-
 __global__ void __launch_bounds__(kThreads) k_quantize(const QuantArgs a) {
-  __shared__ QSmem sm;
+  __shared__ TileSmem sm;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int item = blockIdx.x, dk = a.dk, dv = a.dv;
   const int b = item / a.H, h = item % a.H;
   const int slot = a.slot_idx[b];
   if (slot < 0 || slot >= a.n_slots) {
-    if (tid == 0) atomicOr(a.flag, 1);
+    if (tid == 0) atomicOr(a.flag, SQ_FLAG_BAD_SLOT_BIT);
     return;
   }
   const HeadDesc hd = a.heads[h];
@@ -58,51 +46,15 @@ __global__ void __launch_bounds__(kThreads) k_quantize(const QuantArgs a) {
   if (nonfinite) atomicOr(&sm.misc[1], 1);
   __syncthreads();
   if (sm.misc[1]) {
-    if (tid == 0) atomicOr(a.flag, 2);
+    if (tid == 0) atomicOr(a.flag, SQ_FLAG_NONFINITE_BIT);
     return;
   }
   uint8_t* dst = a.pool + (size_t)slot * a.slot_bytes + hd.off;
-  bool ok;
-  if (hd.pivot_head) {
-    ok = store_pivot_head(S, dst, warp, lane, dk, dv, &sm.misc[0]);
-  } else {
-    const int n_out = a.n_outliers;
-    uint64_t sel = 0;
-    if (n_out > 0) {
-      select_top(S, n_out, warp, lane, dk, dv, rows, sel, sm.wbest, sm.oidx, sm.oval);
-#pragma unroll
-      for (int s = 0; s < kRows; ++s)
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          if ((sel >> (s * 4 + e)) & 1) S[s][e] = 0.f;  // outliers: out of the fit, code 0
-    }
-    fit_scales(S, a.fit_iters, warp, lane, dk, dv, rows, sm.rowW, sm.rowR, sm.rowtmp, sm.red,
-               sm.col);
-    if (n_out > 0 && tid < n_out) {
-      if (__hisinf(__float2half_rn(sm.oval[tid]))) atomicOr(&sm.misc[0], 1);
-    }
-    ok = requant_store_any(mode_of(hd), S, dst, rows, warp, lane, dk, dv, sm.rowR, sm.rowIR,
-                           sm.col, &sm.misc[0]);
-    if (ok && n_out > 0 && tid == 0) {
-      // outlier list in ascending index order (insertion sort of <= 64 entries)
-      uint8_t* o = dst + row_off(rows[dk - 1]) + (size_t)dv * row_width(rows[dk - 1]) / 8;
-      for (int x = 0; x < n_out; ++x) {
-        int bi = -1;
-        for (int y = 0; y < n_out; ++y) {
-          if (sm.oidx[y] < 0) continue;
-          if (bi < 0 || sm.oidx[y] < sm.oidx[bi]) bi = y;
-        }
-        const __half hv = __float2half_rn(sm.oval[bi]);
-        reinterpret_cast<uint16_t*>(o)[2 * x] = (uint16_t)sm.oidx[bi];
-        reinterpret_cast<__half*>(o)[2 * x + 1] = hv;
-        sm.oidx[bi] = -1;
-      }
-    }
-  }
-  if (!ok && tid == 0) atomicOr(a.flag, 4);
-  if (a.side && tid == 0 && h == 0) {  // close the slot's window
-    *reinterpret_cast<int32_t*>(a.side + (size_t)slot * a.side_slot_bytes) = 0;
-  }
+  const bool ok = quantize_tile(S, dst, hd, rows, a.n_outliers, a.fit_iters, warp, lane, dk, dv, sm);
+  if (!ok && tid == 0) atomicOr(a.flag, SQ_FLAG_RANGE_BIT);
+  if (a.side && tid == 0)  // close this head's window
+    *reinterpret_cast<int32_t*>(a.side + (size_t)slot * a.side_slot_bytes +
+                                (size_t)h * a.side_head_bytes) = 0;
 }
 
 // ---------------------------------------------------------------------------------------------

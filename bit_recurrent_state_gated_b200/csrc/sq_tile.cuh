@@ -326,5 +326,183 @@ __device__ __forceinline__ void select_top(const float (&S)[kRows][4], int n, in
   }
 }
 
+
+// ---------------------------------------------------------------------------------------------
+// Shared scratch of the quantize-type kernels (cold quantize, window flush).
+// ---------------------------------------------------------------------------------------------
+constexpr int kMaxOutliers = 64;
+constexpr int kMaxCand = 256;
+
+struct __align__(16) TileSmem {
+  float red[kWarps * 2 * kMaxD];
+  float rowW[kMaxD], rowR[kMaxD], rowIR[kMaxD], rowtmp[kWarps * kRows];
+  float col[N_COL * kMaxD];
+  unsigned long long wbest[kWarps];
+  uint32_t tkey[kThreads];  // per-thread max key
+  uint32_t thr;             // candidate threshold key
+  int ncand;
+  int cand_idx[kMaxCand];
+  float cand_val[kMaxCand];
+  int oidx[kMaxOutliers];
+  float oval[kMaxOutliers];
+  int misc[4];
+};
+
+// Key of an element for the top-n choice: larger |value| first; 0 marks "not eligible".
+__device__ __forceinline__ uint32_t abs_key(float v) { return (__float_as_uint(v) & 0x7fffffffu) + 1u; }
+
+// The n entries of largest |S| among the quantized rows (ties to the lower flat index), exact.
+// Candidate threshold: the n-th largest per-thread maximum is at most the n-th largest element
+// (fewer than n threads can hold an element above the latter), so every selected entry is
+// among the elements at or above it. Falls back to n rounds of CTA arg-max if more than
+// kMaxCand elements reach the threshold. Result in sm.oidx / sm.oval (ascending index) and in
+// `sel` (bit s*4+e of the owning thread). Contains __syncthreads.
+__device__ __forceinline__ void select_top_fast(const float (&S)[kRows][4], int n, int warp,
+                                                int lane, int dk, int dv, const uint32_t* rows,
+                                                uint64_t& sel, TileSmem& sm) {
+  const int tid = threadIdx.x;
+  uint32_t tmax = 0;
+#pragma unroll
+  for (int s = 0; s < kRows; ++s) {
+    const int i = warp * kRows + s;
+    if (i < dk && 4 * lane < dv && row_width(rows[i]) != 16) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) tmax = max(tmax, abs_key(S[s][e]));
+    }
+  }
+  sm.tkey[tid] = tmax;
+  if (tid == 0) sm.ncand = 0;
+  __syncthreads();
+  if (warp == 0) {  // n-th largest of the 256 thread maxima
+    uint32_t v[kThreads / 32];
+#pragma unroll
+    for (int t = 0; t < kThreads / 32; ++t) v[t] = sm.tkey[lane * (kThreads / 32) + t];
+    uint32_t last = 0;
+    for (int r = 0; r < n; ++r) {
+      uint32_t m = 0;
+#pragma unroll
+      for (int t = 0; t < kThreads / 32; ++t) m = max(m, v[t]);
+      const uint32_t wm = __reduce_max_sync(0xffffffffu, m);
+      last = wm;
+      if (wm == 0) break;
+      const uint32_t owner = __ffs(__ballot_sync(0xffffffffu, m == wm)) - 1;
+      if (lane == (int)owner) {
+        bool done = false;
+#pragma unroll
+        for (int t = 0; t < kThreads / 32; ++t)
+          if (!done && v[t] == wm) {
+            v[t] = 0;
+            done = true;
+          }
+      }
+    }
+    if (lane == 0) sm.thr = last;
+  }
+  __syncthreads();
+  const uint32_t thr = sm.thr;
+#pragma unroll
+  for (int s = 0; s < kRows; ++s) {
+    const int i = warp * kRows + s;
+    if (i < dk && 4 * lane < dv && row_width(rows[i]) != 16) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if (abs_key(S[s][e]) >= thr) {
+          const int pos = atomicAdd(&sm.ncand, 1);
+          if (pos < kMaxCand) {
+            sm.cand_idx[pos] = i * dv + 4 * lane + e;
+            sm.cand_val[pos] = S[s][e];
+          }
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (sm.ncand > kMaxCand) {  // many equal values: exact rounds of arg-max
+    select_top(S, n, warp, lane, dk, dv, rows, sel, sm.wbest, sm.oidx, sm.oval);
+  } else {
+    if (warp == 0) {  // top n of the candidates by (|v| desc, index asc)
+      const int nc = sm.ncand;
+      for (int r = 0; r < n; ++r) {
+        unsigned long long best = 0;
+        int bpos = -1;
+        for (int p = lane; p < nc; p += 32) {
+          const int idx = sm.cand_idx[p];
+          if (idx < 0) continue;
+          const unsigned long long key =
+              ((unsigned long long)abs_key(sm.cand_val[p]) << 32) | (0xffffffffu - (uint32_t)idx);
+          if (key > best) {
+            best = key;
+            bpos = p;
+          }
+        }
+        unsigned long long wb = best;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          const unsigned long long other = __shfl_xor_sync(0xffffffffu, wb, o);
+          wb = other > wb ? other : wb;
+        }
+        if (best == wb && bpos >= 0 && wb != 0) {
+          sm.oidx[r] = sm.cand_idx[bpos];
+          sm.oval[r] = sm.cand_val[bpos];
+          sm.cand_idx[bpos] = -1;
+        }
+        __syncwarp();
+      }
+    }
+    __syncthreads();
+    sel = 0;
+    for (int r = 0; r < n; ++r) {
+      const int idx = sm.oidx[r], wi = idx / dv, wj = idx % dv;
+      if (wi / kRows == warp && wj / 4 == lane) sel |= 1ull << ((wi % kRows) * 4 + wj % 4);
+    }
+  }
+  __syncthreads();
+  if (tid == 0) {  // ascending index order
+    for (int x = 1; x < n; ++x) {
+      const int ki = sm.oidx[x];
+      const float kv = sm.oval[x];
+      int y = x - 1;
+      while (y >= 0 && sm.oidx[y] > ki) {
+        sm.oidx[y + 1] = sm.oidx[y];
+        sm.oval[y + 1] = sm.oval[y];
+        --y;
+      }
+      sm.oidx[y + 1] = ki;
+      sm.oval[y + 1] = kv;
+    }
+  }
+  __syncthreads();
+}
+
+// Quantize a register tile into the head block at dst: the n_out compensation entries (if
+// any) are chosen and stored in fp16, the rest is fit and packed. Returns false (nothing
+// stored) on an fp16 range overflow. Contains __syncthreads; sm.misc[0] must be 0 on entry.
+__device__ __forceinline__ bool quantize_tile(float (&S)[kRows][4], uint8_t* dst,
+                                              const HeadDesc& hd, const uint32_t* rows,
+                                              int n_out, int fit_iters, int warp, int lane,
+                                              int dk, int dv, TileSmem& sm) {
+  if (hd.pivot_head) return store_pivot_head(S, dst, warp, lane, dk, dv, &sm.misc[0]);
+  if (n_out > 0) {
+    uint64_t sel = 0;
+    select_top_fast(S, n_out, warp, lane, dk, dv, rows, sel, sm);
+#pragma unroll
+    for (int s = 0; s < kRows; ++s)
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if ((sel >> (s * 4 + e)) & 1) S[s][e] = 0.f;  // outliers: out of the fit, code 0
+    if ((int)threadIdx.x < n_out && __hisinf(__float2half_rn(sm.oval[threadIdx.x])))
+      atomicOr(&sm.misc[0], 1);
+  }
+  fit_scales(S, fit_iters, warp, lane, dk, dv, rows, sm.rowW, sm.rowR, sm.rowtmp, sm.red, sm.col);
+  const bool ok = requant_store_any(mode_of(hd), S, dst, rows, warp, lane, dk, dv, sm.rowR,
+                                    sm.rowIR, sm.col, &sm.misc[0]);
+  if (ok && n_out > 0 && (int)threadIdx.x < n_out) {
+    uint8_t* o = dst + row_off(rows[dk - 1]) + (size_t)dv * row_width(rows[dk - 1]) / 8;
+    const int x = threadIdx.x;
+    reinterpret_cast<uint16_t*>(o)[2 * x] = (uint16_t)sm.oidx[x];
+    reinterpret_cast<__half*>(o)[2 * x + 1] = __float2half_rn(sm.oval[x]);
+  }
+  return ok;
+}
 }  // namespace tile
 }  // namespace sq
