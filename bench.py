@@ -45,7 +45,7 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="gdn", choices=["tiny", "gdn", "kda", "pool"])
+    ap.add_argument("--workload", default="gdn", choices=["tiny", "gdn", "kda", "pool", "window"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
@@ -56,12 +56,24 @@ def parse():
 
 def algorithmic_bytes(wl: W.Workload, slot_bytes: int) -> dict:
     """Bytes one request-step must move: the packed state (codes, scales, fp16 units) read and
-    written, q/k/v read, alpha/beta read, o written, the slot index read."""
+    written, q/k/v read, alpha/beta read, o written, the slot index read. Windowed layouts read
+    the frozen block every token and write it once per window; their low-rank side state
+    (the cumulative gate and one (k_hat, b) pair per token, fp32) is counted as `side`."""
     esz = 2 if wl.io_dtype == W.IO_BF16 else 4
-    H = wl.n_heads
-    state = 2 * slot_bytes
-    io = H * (2 * wl.d_k + wl.d_v) * esz + H * wl.alpha_width * 4 + H * 4 + H * wl.d_v * 4 + 4
-    return {"state": state, "io": io, "total": state + io}
+    H, dk, dv = wl.n_heads, wl.d_k, wl.d_v
+    io = H * (2 * dk + dv) * esz + H * wl.alpha_width * 4 + H * 4 + H * dv * 4 + 4
+    if wl.window <= 1:
+        state, side = 2 * slot_bytes, 0
+    else:
+        Wn = wl.window
+        state = slot_bytes + slot_bytes / Wn
+        term = 4 * (dk + dv)
+        # per head and window: token t reads t terms and (t > 0) the gate; tokens 0..W-2 write
+        # a term, the gate and the count
+        reads = sum(t * term + (4 * dk if t else 0) for t in range(Wn))
+        writes = (Wn - 1) * (term + 4 * dk + 4)
+        side = H * (reads + writes) / Wn
+    return {"state": state, "side": side, "io": io, "total": state + side + io}
 
 
 def peaks() -> tuple[float, str]:
@@ -171,8 +183,10 @@ def oracle_rate(wl: W.Workload, seconds: float, t0: int = 0):
     import oracle
     threads = oracle.default_threads()
     n_req = max(1, min(wl.batch, threads))
-    lay = oracle.Layout(wl.n_heads, wl.d_k, wl.d_v, wl.unit, wl.gate, wl.fit_iters)
+    lay = oracle.Layout(wl.n_heads, wl.d_k, wl.d_v, wl.unit, wl.gate, wl.fit_iters, wl.window,
+                        wl.n_outliers)
     pool = oracle.Pool(lay, wl.bits(), n_req)
+    step = pool.window_step if wl.window > 1 else pool.decode_step
     si = np.arange(n_req, dtype=np.int32)
     pool.quantize(si, wl.initial_state(wl.slot_idx()[:n_req]))
     sets = []
@@ -183,7 +197,7 @@ def oracle_rate(wl: W.Workload, seconds: float, t0: int = 0):
     while busy < seconds:  # only the oracle's own calls are timed
         xs = sets[n % len(sets)]
         ts = time.perf_counter()
-        pool.decode_step(si, xs["q"], xs["k"], xs["v"], xs["alpha"], xs["beta"], threads=threads)
+        step(si, xs["q"], xs["k"], xs["v"], xs["alpha"], xs["beta"], threads=threads)
         busy += time.perf_counter() - ts
         done += n_req
         n += 1
@@ -318,6 +332,7 @@ def run_ours(args, info):
             "io": "bf16" if wl.io_dtype == W.IO_BF16 else "f32", "fit_iters": wl.fit_iters,
             "state_bytes_per_request": pool.slot_bytes,
             "algorithmic_bytes_per_request_step": ab["total"],
+            "window": wl.window, "compensation_entries_per_head": wl.n_outliers,
             "l2": "flushed before every timed step (write, then read, 256 MB)",
             "parallelism": f"dp{info.world} (requests partitioned, no collective)",
         },
@@ -325,7 +340,8 @@ def run_ours(args, info):
                      "frac": achieved / peak, "traffic": traffic,
                      "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)"
                      if peak_kind == "measured" else "fallback 6.65 TB/s",
-                     "kernel": "k_decode", "mean_launch_us": mean_launch_s * 1e6},
+                     "kernel": "k_window_step" if wl.window > 1 else "k_decode",
+                     "mean_launch_us": mean_launch_s * 1e6},
         "e2e": {"value": total_req_steps / (e2e_ms / 1e3), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": args.steps,
