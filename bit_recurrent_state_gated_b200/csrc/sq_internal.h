@@ -45,6 +45,7 @@ struct StepArgs {
   int32_t H, dk, dv, fit_iters;
   int32_t per_row;       // 1: key-row units (the row table is staged with each head block)
   uint32_t stage_bytes;  // smem bytes reserved for one staged head block
+  int32_t n_stages;      // staged items in flight (set by the decode launcher)
   int32_t* flag;
   // windowed variant
   uint8_t* side;          // side region base (n_slots * side_slot_bytes)
@@ -69,7 +70,7 @@ struct QuantArgs {
   int64_t side_slot_bytes, side_head_bytes;
 };
 
-// Launchers (sq_kernels.cu). Return cudaSuccess or the launch error.
+// Launchers (sq_decode.cu, sq_quant.cu, sq_window.cu). Return cudaSuccess or the launch error.
 cudaError_t launch_decode(const StepArgs& a, int gate, int io, bool want_state, int num_sms,
                           cudaStream_t st);
 cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t st);

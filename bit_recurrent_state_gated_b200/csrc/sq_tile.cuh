@@ -139,7 +139,7 @@ __device__ __forceinline__ bool requant_store(const float (&S)[kRows][4], uint8_
       if (q_of_width(row_width(rows[i])) > 0) {
         const __half r16 = __float2half_rn(rowR[i]);
         if (__hisinf(r16)) atomicOr(bad, 1);
-        ir = __frcp_rn(__half2float(r16));
+        ir = rcp_f16val(__half2float(r16));
       }
       rowIR[i] = ir;
     }
@@ -147,7 +147,7 @@ __device__ __forceinline__ bool requant_store(const float (&S)[kRows][4], uint8_
   if (t < dv) {
     const __half c16 = __float2half_rn(col[COL_X * kMaxD + t]);
     if (__hisinf(c16)) atomicOr(bad, 1);
-    col[COL_IC16 * kMaxD + t] = __frcp_rn(__half2float(c16));
+    col[COL_IC16 * kMaxD + t] = rcp_f16val(__half2float(c16));
   } else if (t < kMaxD) {
     col[COL_IC16 * kMaxD + t] = 0.f;
   }
