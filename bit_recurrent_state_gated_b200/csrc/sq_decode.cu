@@ -195,7 +195,8 @@ __device__ __forceinline__ float4 max8(const float* red, int lane) {
 template <int MODE, bool FULL>
 __device__ __forceinline__ void pass_a(const Ctx<FULL>& c) {
   const Geo<MODE> geo(c);
-  float2 U0 = f2(0.f, 0.f), U1 = U0, P0 = U0, P1 = U0;
+  // two accumulator sets (even / odd rows) halve the dependent-add chains
+  float2 U0 = f2(0.f, 0.f), U1 = U0, P0 = U0, P1 = U0, U2 = U0, U3 = U0, P2 = U0, P3 = U0;
   if (c.wact()) {
     float4 icv = make_float4(1.f, 1.f, 1.f, 1.f);
     if (MODE == MODE_ROWS && c.act()) {  // 1/c16 of the lane's columns, for fp16 rows
@@ -206,36 +207,45 @@ __device__ __forceinline__ void pass_a(const Ctx<FULL>& c) {
     }
 #pragma unroll 1
     for (int ch = 0; ch < kChunks; ++ch) {
-      float v[16];
+      float2 v[8];
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
         const int i = c.row0() + 4 * ch + r;
-        float* x = v + 4 * r;
+        float2 x01 = f2(0.f, 0.f), x23 = x01;
         const int b = geo.width(i);
         if (c.act()) {
           const uint8_t* row = c.blk + geo.off(i);
           if constexpr (MODE == MODE_ROWS)
-            unpack4_rt(b, row, c.lane, x);
+            unpack4x2_rt(b, row, c.lane, x01, x23);
           else
-            unpack4<MODE>(row, c.lane, x);
-        } else {
-          x[0] = x[1] = x[2] = x[3] = 0.f;
+            unpack4x2<MODE>(row, c.lane, x01, x23);
         }
-        float2 x01 = f2(x[0], x[1]), x23 = f2(x[2], x[3]);
         if (MODE == MODE_ROWS && b == 16) {  // fp16 row inside a scaled head: x = value / c_j
           x01 = __fmul2_rn(x01, lo(icv));
           x23 = __fmul2_rn(x23, hi(icv));
-          x[0] = x01.x, x[1] = x01.y, x[2] = x23.x, x[3] = x23.y;
         }
+        v[2 * r] = x01;
+        v[2 * r + 1] = x23;
         const float4 g = c.rowG()[i];  // (gk, gk, gq, gq)
-        U0 = __ffma2_rn(x01, lo(g), U0);
-        U1 = __ffma2_rn(x23, lo(g), U1);
-        P0 = __ffma2_rn(x01, hi(g), P0);
-        P1 = __ffma2_rn(x23, hi(g), P1);
+        if (r & 1) {
+          U2 = __ffma2_rn(x01, lo(g), U2);
+          U3 = __ffma2_rn(x23, lo(g), U3);
+          P2 = __ffma2_rn(x01, hi(g), P2);
+          P3 = __ffma2_rn(x23, hi(g), P3);
+        } else {
+          U0 = __ffma2_rn(x01, lo(g), U0);
+          U1 = __ffma2_rn(x23, lo(g), U1);
+          P0 = __ffma2_rn(x01, hi(g), P0);
+          P1 = __ffma2_rn(x23, hi(g), P1);
+        }
       }
-      tmem_st16(c.tm + 16 * ch, v);
+      tmem_st16x2(c.tm + 16 * ch, v);
     }
   }
+  U0 = __fadd2_rn(U0, U2);
+  U1 = __fadd2_rn(U1, U3);
+  P0 = __fadd2_rn(P0, P2);
+  P1 = __fadd2_rn(P1, P3);
   float* red = sp<float>(OFF_REDA) + c.warp * 2 * kMaxD + 4 * c.lane;
   *reinterpret_cast<float4*>(red) = make_float4(U0.x, U0.y, U1.x, U1.y);
   *reinterpret_cast<float4*>(red + kMaxD) = make_float4(P0.x, P0.y, P1.x, P1.y);
@@ -250,18 +260,17 @@ __device__ __forceinline__ void pass_b(const Ctx<FULL>& c, const float4& cv, con
   if (c.wact()) {
 #pragma unroll 1
     for (int ch = 0; ch < kChunks; ++ch) {
-      float v[16];
-      tmem_ld16(c.tm + 16 * ch, v);
+      float2 v[8];
+      tmem_ld16x2(c.tm + 16 * ch, v);
       float rm[4];
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
         const int i = c.row0() + 4 * ch + r;
         const float4 u = c.rowU()[i];  // (A, A, k, k)
-        const float2 s0 = __ffma2_rn(f2(v[4 * r], v[4 * r + 1]), __fmul2_rn(lo(u), lo(cv)),
-                                     __fmul2_rn(hi(u), lo(bv)));
-        const float2 s1 = __ffma2_rn(f2(v[4 * r + 2], v[4 * r + 3]), __fmul2_rn(lo(u), hi(cv)),
-                                     __fmul2_rn(hi(u), hi(bv)));
-        v[4 * r] = s0.x, v[4 * r + 1] = s0.y, v[4 * r + 2] = s1.x, v[4 * r + 3] = s1.y;
+        const float2 s0 = __ffma2_rn(v[2 * r], __fmul2_rn(lo(u), lo(cv)), __fmul2_rn(hi(u), lo(bv)));
+        const float2 s1 = __ffma2_rn(v[2 * r + 1], __fmul2_rn(lo(u), hi(cv)), __fmul2_rn(hi(u), hi(bv)));
+        v[2 * r] = s0;
+        v[2 * r + 1] = s1;
         if (fit) rm[r] = warp_max_nonneg(fmaxf(max3abs(s0.x, s0.y, s1.x), fabsf(s1.y)));
         if (check16 == 1 || (check16 == 2 && row_width(c.rowtab()[i]) == 16))  // RN16 -> inf
           if (c.act()) of |= !(fmaxf(max3abs(s0.x, s0.y, s1.x), fabsf(s1.y)) < 65520.f);
@@ -269,7 +278,7 @@ __device__ __forceinline__ void pass_b(const Ctx<FULL>& c, const float4& cv, con
           *reinterpret_cast<float4*>(s_new + (size_t)i * c.dv() + 4 * c.lane) =
               make_float4(s0.x, s0.y, s1.x, s1.y);
       }
-      tmem_st16(c.tm + 16 * ch, v);
+      tmem_st16x2(c.tm + 16 * ch, v);
       if (fit && c.lane == 0)
         *reinterpret_cast<float4*>(c.rowtmp() + 4 * ch) = make_float4(rm[0], rm[1], rm[2], rm[3]);
     }
@@ -307,28 +316,36 @@ __device__ __forceinline__ float row_scales(const Ctx<FULL>& c, int mode, bool c
 // Column pass: max_i |S_ij| w_i over the warp's rows, into red[warp].
 template <bool FULL>
 __device__ __forceinline__ void col_pass(const Ctx<FULL>& c, float* red) {
-  float cm0 = 0.f, cm1 = 0.f, cm2 = 0.f, cm3 = 0.f;
+  float cm0 = 0.f, cm1 = 0.f, cm2 = 0.f, cm3 = 0.f, cn0 = 0.f, cn1 = 0.f, cn2 = 0.f, cn3 = 0.f;
   if (c.wact()) {
     const float4* w2 = reinterpret_cast<const float4*>(c.rowW2() + c.row0());
 #pragma unroll 1
     for (int ch = 0; ch < kChunks; ++ch) {
-      float v[16];
-      tmem_ld16(c.tm + 16 * ch, v);
+      float2 v[8];
+      tmem_ld16x2(c.tm + 16 * ch, v);
 #pragma unroll
       for (int r = 0; r < 4; r += 2) {
         const float4 ww = w2[2 * ch + r / 2];  // (w_s, w_s, w_s+1, w_s+1)
-        const float2 a0 = __fmul2_rn(f2(v[4 * r], v[4 * r + 1]), lo(ww));
-        const float2 a1 = __fmul2_rn(f2(v[4 * r + 2], v[4 * r + 3]), lo(ww));
-        const float2 b0 = __fmul2_rn(f2(v[4 * r + 4], v[4 * r + 5]), hi(ww));
-        const float2 b1 = __fmul2_rn(f2(v[4 * r + 6], v[4 * r + 7]), hi(ww));
-        cm0 = max3abs(cm0, a0.x, b0.x);
-        cm1 = max3abs(cm1, a0.y, b0.y);
-        cm2 = max3abs(cm2, a1.x, b1.x);
-        cm3 = max3abs(cm3, a1.y, b1.y);
+        const float2 a0 = __fmul2_rn(v[2 * r], lo(ww));
+        const float2 a1 = __fmul2_rn(v[2 * r + 1], lo(ww));
+        const float2 b0 = __fmul2_rn(v[2 * r + 2], hi(ww));
+        const float2 b1 = __fmul2_rn(v[2 * r + 3], hi(ww));
+        if (r == 0) {
+          cm0 = max3abs(cm0, a0.x, b0.x);
+          cm1 = max3abs(cm1, a0.y, b0.y);
+          cm2 = max3abs(cm2, a1.x, b1.x);
+          cm3 = max3abs(cm3, a1.y, b1.y);
+        } else {
+          cn0 = max3abs(cn0, a0.x, b0.x);
+          cn1 = max3abs(cn1, a0.y, b0.y);
+          cn2 = max3abs(cn2, a1.x, b1.x);
+          cn3 = max3abs(cn3, a1.y, b1.y);
+        }
       }
     }
   }
-  *reinterpret_cast<float4*>(red + c.warp * kMaxD + 4 * c.lane) = make_float4(cm0, cm1, cm2, cm3);
+  *reinterpret_cast<float4*>(red + c.warp * kMaxD + 4 * c.lane) =
+      make_float4(fmaxf(cm0, cn0), fmaxf(cm1, cn1), fmaxf(cm2, cn2), fmaxf(cm3, cn3));
 }
 
 // Row pass of a later alternation: row maxima of |S_ij| v_j into rowtmp.
@@ -337,13 +354,13 @@ __device__ __forceinline__ void row_pass(const Ctx<FULL>& c, const float4& icv) 
   if (c.wact()) {
 #pragma unroll 1
     for (int ch = 0; ch < kChunks; ++ch) {
-      float v[16];
-      tmem_ld16(c.tm + 16 * ch, v);
+      float2 v[8];
+      tmem_ld16x2(c.tm + 16 * ch, v);
       float rm[4];
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
-        const float2 p = __fmul2_rn(f2(v[4 * r], v[4 * r + 1]), lo(icv));
-        const float2 q = __fmul2_rn(f2(v[4 * r + 2], v[4 * r + 3]), hi(icv));
+        const float2 p = __fmul2_rn(v[2 * r], lo(icv));
+        const float2 q = __fmul2_rn(v[2 * r + 1], hi(icv));
         rm[r] = warp_max_nonneg(fmaxf(max3abs(p.x, p.y, q.x), fabsf(q.y)));
       }
       if (c.lane == 0)
@@ -380,21 +397,21 @@ __device__ __forceinline__ void requant(const Ctx<FULL>& c, uint8_t* dst, const 
   if (!c.wact()) return;
 #pragma unroll 1
   for (int ch = 0; ch < kChunks; ++ch) {
-    float v[16];
-    tmem_ld16(c.tm + 16 * ch, v);
+    float2 v[8];
+    tmem_ld16x2(c.tm + 16 * ch, v);
 #pragma unroll
     for (int r2 = 0; r2 < 4; ++r2) {
       const int i = c.row0() + 4 * ch + r2;
       uint8_t* row = dst + geo.off(i);
       const int b = geo.width(i);
       if (MODE == MODE_ROWS && b == 16) {
-        store4_f16(row, c.lane, v + 4 * r2, c.act());
+        store4_f16x2(row, c.lane, v[2 * r2], v[2 * r2 + 1], c.act());
       } else {
         const float2 ir = c.rowIR2()[i];
         const float mgv = kMagic + (float)(1 << (b - 1));
         const float2 mg = f2(mgv, mgv);
-        const float2 y0 = __ffma2_rn(__fmul2_rn(f2(v[4 * r2], v[4 * r2 + 1]), ir), ic01, mg);
-        const float2 y1 = __ffma2_rn(__fmul2_rn(f2(v[4 * r2 + 2], v[4 * r2 + 3]), ir), ic23, mg);
+        const float2 y0 = __ffma2_rn(__fmul2_rn(v[2 * r2], ir), ic01, mg);
+        const float2 y1 = __ffma2_rn(__fmul2_rn(v[2 * r2 + 1], ir), ic23, mg);
         const float y[4] = {y0.x, y0.y, y1.x, y1.y};
         if constexpr (MODE == MODE_ROWS) {
           switch (b) {
@@ -418,10 +435,11 @@ __device__ __forceinline__ void store_pivot(const Ctx<FULL>& c, uint8_t* dst) {
   const Geo<MODE_PIVOT> geo(c);
 #pragma unroll 1
   for (int ch = 0; ch < kChunks; ++ch) {
-    float v[16];
-    tmem_ld16(c.tm + 16 * ch, v);
+    float2 v[8];
+    tmem_ld16x2(c.tm + 16 * ch, v);
 #pragma unroll
-    for (int r = 0; r < 4; ++r) store4_f16(dst + geo.off(c.row0() + 4 * ch + r), c.lane, v + 4 * r, c.act());
+    for (int r = 0; r < 4; ++r)
+      store4_f16x2(dst + geo.off(c.row0() + 4 * ch + r), c.lane, v[2 * r], v[2 * r + 1], c.act());
   }
 }
 
@@ -748,18 +766,21 @@ cudaError_t launch_t(const StepArgs& a, int num_sms, cudaStream_t st) {
   StepArgs b = a;
   uint32_t smem_bytes = 0;
   int per_sm = 0;
-  cudaError_t e = cudaSuccess;
-  for (int nst = 2; nst >= 1; --nst) {
+  for (int nst = 2; nst >= 1; --nst) {  // the most CTAs per SM, then the most stages
     const DPlan P(a.dk, a.dv, IO, GATE, a.per_row, a.stage_bytes, a.H, nst);
-    smem_bytes = P.total > 47u * 1024u ? P.total : 47u * 1024u;
-    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
+    const uint32_t sb = P.total > 47u * 1024u ? P.total : 47u * 1024u;
+    int n = 0;
+    const cudaError_t e = resident_ctas(reinterpret_cast<const void*>(fn), sb, &n);
     if (e != cudaSuccess) return e;
-    e = resident_ctas(reinterpret_cast<const void*>(fn), smem_bytes, &per_sm);
-    if (e != cudaSuccess) return e;
-    b.n_stages = nst;
-    if (per_sm >= 3) break;
+    if (n > kMaxCtasPerSm) n = kMaxCtasPerSm;
+    if (n > per_sm) {
+      per_sm = n;
+      smem_bytes = sb;
+      b.n_stages = nst;
+    }
   }
-  if (per_sm > kMaxCtasPerSm) per_sm = kMaxCtasPerSm;
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
+  if (e != cudaSuccess) return e;
   const int items = a.batch * a.H;
   int grid = num_sms * per_sm;
   if (grid > items) grid = items;
