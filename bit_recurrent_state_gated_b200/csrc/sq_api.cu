@@ -15,12 +15,14 @@ struct sq_pool {
   std::vector<uint8_t> bits;  // unit widths (16 = pivot)
   std::vector<sq::HeadDesc> heads;
   std::vector<uint32_t> rows;  // [H][d_k] (offset << 8) | width
+  std::vector<uint32_t> srows;  // key-row units: [H][d_k] descriptors, rows grouped by width
   size_t slot_bytes = 0, side_slot_bytes = 0, side_head_bytes = 0;
   uint32_t max_head_bytes = 0;
   uint8_t* base = nullptr;  // caller's buffer
   std::vector<int32_t> order;  // heads sorted by width (pivot heads last)
   sq::HeadDesc* d_heads = nullptr;
   uint32_t* d_rows = nullptr;
+  uint32_t* d_srows = nullptr;
   int32_t* d_order = nullptr;
   int32_t* d_flag = nullptr;
   int device = 0, num_sms = 0;
@@ -89,6 +91,25 @@ sq_status plan(const sq_layout* L, const uint8_t* bits, const uint8_t* pivot_mas
   }
   P->slot_bytes = off;
   P->max_head_bytes = maxb;
+  if (L->unit == SQ_UNIT_KEY_ROW) {
+    // Processing order of the decode kernel: each head's rows grouped by width (stable), so
+    // that row pairs and four-row chunks almost always share one width.
+    P->srows.assign((size_t)H * dk, 0);
+    for (int h = 0; h < H; ++h) {
+      std::vector<int> idx(dk);
+      for (int i = 0; i < dk; ++i) idx[i] = i;
+      const uint32_t* rt = &P->rows[(size_t)h * dk];
+      std::stable_sort(idx.begin(), idx.end(), [&](int x, int y) {
+        return sq::row_width(rt[x]) < sq::row_width(rt[y]);
+      });
+      for (int p = 0; p < dk; ++p) {
+        const uint32_t d = rt[idx[p]];
+        if (sq::row_off(d) >= (1u << 16)) return SQ_ERR_INVALID_ARG;
+        P->srows[(size_t)h * dk + p] =
+            (uint32_t)idx[p] << 24 | sq::row_off(d) << 8 | (uint32_t)sq::row_width(d);
+      }
+    }
+  }
   P->order.resize(H);
   for (int h = 0; h < H; ++h) P->order[h] = h;
   std::stable_sort(P->order.begin(), P->order.end(), [&](int x, int y) {
@@ -138,6 +159,7 @@ sq::StepArgs step_args(sq_pool* p, const int32_t* slot_idx, int32_t batch, const
   a.s_new = s_new;
   a.heads = p->d_heads;
   a.rows = p->d_rows;
+  a.srows = p->d_srows;
   a.order = p->d_order;
   a.H = p->L.n_heads;
   a.dk = p->L.d_k;
@@ -230,6 +252,11 @@ sq_status sq_state_pool_create(const sq_layout* layout, const uint8_t* bits_map,
   }
   if (e == cudaSuccess) e = cudaMalloc(&p->d_heads, sizeof(sq::HeadDesc) * p->heads.size());
   if (e == cudaSuccess) e = cudaMalloc(&p->d_rows, sizeof(uint32_t) * p->rows.size());
+  if (e == cudaSuccess && !p->srows.empty())
+    e = cudaMalloc(&p->d_srows, sizeof(uint32_t) * p->srows.size());
+  if (e == cudaSuccess && !p->srows.empty())
+    e = cudaMemcpy(p->d_srows, p->srows.data(), sizeof(uint32_t) * p->srows.size(),
+                   cudaMemcpyHostToDevice);
   if (e == cudaSuccess) e = cudaMalloc(&p->d_flag, sizeof(int32_t));
   if (e == cudaSuccess) e = cudaMalloc(&p->d_order, sizeof(int32_t) * p->order.size());
   if (e == cudaSuccess)
@@ -245,6 +272,7 @@ sq_status sq_state_pool_create(const sq_layout* layout, const uint8_t* bits_map,
   if (e != cudaSuccess) {
     cudaFree(p->d_heads);
     cudaFree(p->d_rows);
+    cudaFree(p->d_srows);
     cudaFree(p->d_flag);
     cudaFree(p->d_order);
     delete p;
@@ -258,6 +286,7 @@ sq_status sq_state_pool_destroy(sq_pool* pool) {
   if (!pool) return SQ_OK;
   cudaFree(pool->d_heads);
   cudaFree(pool->d_rows);
+  cudaFree(pool->d_srows);
   cudaFree(pool->d_flag);
   cudaFree(pool->d_order);
   delete pool;

@@ -2,42 +2,54 @@
 //
 // STEPQuant explainer, experimental-setup paragraph: at every decode step the packed state is
 // unpacked, updated and written back by one fused kernel, and the row / column scales are
-// refit on the updated state. Per (request, head) item:
-//   the packed head block and q, k, v (alpha) arrive in shared memory by bulk copy; unpack
-//   exact codes x; U_j = sum_i x_ij A_i k_i and P_j = sum_i x_ij A_i q_i (A_i = alpha_i r16_i,
-//   so S'^T k = c * U); b = beta (v - c U); o = c P + b (k.q); M_new_ij = x_ij (A_i c_j) +
-//   k_i b_j; refit the dual-axis scales by alternating max-abs passes; requantize, repack and
-//   store in place.
+// refit on the updated state. Per (request, head) item, with x the exact integer codes of the
+// packed head, A_i = alpha_i r16_i and c_j = c16_j (so S'_ij = A_i x_ij c_j):
+//   pass A  unpack x; U_j = sum_i x_ij A_i k_i, P_j = sum_i x_ij A_i q_i (S'^T k = c U);
+//   ----    b = beta (v - c U);  o = c P + b (k.q)
+//   pass B  M_new_ij = x_ij (A_i c_j) + k_i b_j, row maxima of |M_new|
+//   fit     alternating row / column max-abs passes (fit_iters alternations)
+//   pass Q  requantize, repack and store in place.
 //
-// Where the tile lives. Each thread owns 16 key rows x 4 value columns of the 128 x 128 fp32
-// tile (warp w: rows 16w..16w+15, lane l: columns 4l..4l+3), and keeps its 64 values in the
-// SM's tensor memory, not in registers: the CTA allocates 128 tensor-memory columns, and
-// thread t of warp w uses columns 64 (w / 4) .. + 63 of lane 32 (w % 4) + t. Every pass over
-// the tile streams 4-row chunks (16 values) through registers with one tcgen05.ld and, where
-// the pass changes the tile, one tcgen05.st. With the tile out of the register file a CTA
-// needs few registers, so three or four CTAs share an SM (four tiles fill the 512 columns)
-// and each one's barrier and load latency is covered by the others' passes; the passes are
-// loops, which keeps the instruction footprint small.
+// Mapping. A CTA of four warps handles one item at a time; warp w owns 32 key rows, lane l
+// owns value columns 4l .. 4l+3, so every thread holds 32 x 4 fp32 state values. They live in
+// the SM's tensor memory: the CTA allocates 128 columns and thread t of warp w keeps its values
+// in columns 0..127 of lane 32 w + t, written and read 16 at a time (four rows) with tcgen05.st
+// / tcgen05.ld. With the tile out of the register file four CTAs (four items) share an SM and
+// fill its 512 tensor-memory columns. Rows are processed in pairs: a register pair holds the
+// same column of two rows, so one shared-memory broadcast serves two rows' factors and the
+// packed fp32x2 instructions do two elements at a time. Key-row units are processed in an
+// order that groups rows of equal width (a per-head permutation fixed when the pool is made),
+// so almost every row pair and four-row chunk has one width.
 //
-// Row work stays inside a warp (warp redux for row maxima, per-row factors in warp-private
-// shared memory); column sums and maxima combine the 8 warps' partials. Three CTA barriers per
-// item (fit_iters = 2). One lane issues the bulk copies of the next item into the single
-// stage right after the first barrier, so the copy overlaps the item's remaining passes.
+// Row work stays inside a warp (redux for row maxima; per-row scalars computed by the lane
+// whose index is the row); column sums and maxima combine the four warps' partials after a CTA
+// barrier, three per item for fit_iters = 2. Tensor-memory loads are issued one chunk ahead of
+// their use. The packed head block and q, k, v (alpha, row table) of the next item arrive by
+// bulk copies issued right after the current item's first barrier, when the single staging
+// buffer is free again.
 //
 // Arithmetic: the refit follows the oracle's rule step for step with correctly rounded
 // operations (r_i = max(m_i / Q_i, 2^-14), w_i = 1/(r_i Q_i), c_j = max(max_i |S_ij| w_i,
 // 2^-14), v_j = 1/c_j, fp16 rounding once); the code multipliers 1/r16 and 1/c16 are correctly
-// rounded as well. The state is the GPU's own fp32 update (fused multiply-adds), so its scales
-// and codes are compared with the oracle's within the stated agreement.
+// rounded as well. Codes need no clamp: the fit makes every |S_ij| w_i <= c_j, so the quotient
+// S_ij / (r16_i c16_j) is at most Q (1 + 2^-10) in magnitude, less than Q + 1/2 for Q <= 127.
+// The state is the GPU's own fp32 update (fused multiply-adds), so its scales and codes are
+// compared with the oracle's within the stated agreement.
 #include "sq_tile.cuh"
 
 namespace sq {
 namespace {
-using namespace tile;
+using tile::ld_io;
+using tile::q_of_width;
+using tile::round16;
 
-constexpr uint32_t kTmemCols = 128;  // 8 warps x 32 lanes x 64 values = 128 lanes x 128 columns
-constexpr int kMaxCtasPerSm = 4;     // 4 x 128 columns: the SM's whole tensor memory
-constexpr int kChunks = kRows / 4;   // 4-row chunks per warp and pass
+constexpr int kW = 4;                 // warps per CTA
+constexpr int kT = 32 * kW;           // threads per CTA
+constexpr int kRW = 32;               // key rows per warp
+constexpr int kMaxCh = kRW / 4;       // four-row chunks per warp
+constexpr uint32_t kTmemCols = 128;   // 32 rows x 4 columns per thread
+constexpr int kMaxCtasPerSm = 4;      // 4 x 128 columns: the SM's whole tensor memory
+constexpr int MODE_ROWS = 0, MODE_PIVOT = 16;
 
 struct StageHdr {
   int32_t valid, slot, b, h;
@@ -53,34 +65,36 @@ struct Meta {
   int32_t pad;
 };
 
-// Flag words of an item: [0] non-finite input, [1] fp16 range overflow.
 enum { F_INPUT = 0, F_RANGE = 1 };
 
-// Shared memory: fixed-size arrays at compile-time offsets, then the stage and the head table.
-constexpr uint32_t OFF_BAR = 0;                                   // stage mbarriers (<= 2)
-constexpr uint32_t OFF_TMEM = 16;                                 // tensor-memory base address
-constexpr uint32_t OFF_FLAGS = 32;                                // [4 items][4] ints
-constexpr uint32_t OFF_META = 96;                                 // Meta
-constexpr uint32_t OFF_REDA = 112;                                // [8 warps][2][128] U, P
-constexpr uint32_t OFF_REDC = OFF_REDA + kWarps * 2 * kMaxD * 4;  // [2][8 warps][128] col maxima
-constexpr uint32_t OFF_ROWG = OFF_REDC + 2 * kWarps * kMaxD * 4;  // float4 (gk, gk, gq, gq)
-constexpr uint32_t OFF_ROWU = OFF_ROWG + kMaxD * 16;              // float4 (A, A, k, k)
-constexpr uint32_t OFF_ROWW2 = OFF_ROWU + kMaxD * 16;             // float2 (w, w)
-constexpr uint32_t OFF_ROWIR2 = OFF_ROWW2 + kMaxD * 8;            // float2 (1/r16, 1/r16)
-constexpr uint32_t OFF_ROWTAB = OFF_ROWIR2 + kMaxD * 8;           // row descriptors
-constexpr uint32_t OFF_ROWTMP = OFF_ROWTAB + kMaxD * 4;           // per warp: 16 maxima / r16
-constexpr uint32_t OFF_COLC = OFF_ROWTMP + kWarps * kRows * 4;    // c16 of the item, as float
-constexpr uint32_t OFF_COLV = OFF_COLC + kMaxD * 4;               // v of the item, as float
-constexpr uint32_t OFF_KQP = OFF_COLV + kMaxD * 4;                // per-warp partials of k.q
-constexpr uint32_t OFF_STAGE = OFF_KQP + kWarps * 4;              // multiple of 16
-static_assert(OFF_STAGE % 16 == 0 && OFF_REDA % 16 == 0, "16-byte aligned regions");
+// Fixed shared memory (byte offsets).
+constexpr uint32_t S_BAR = 0;                 // stage mbarrier
+constexpr uint32_t S_TMEM = 8;                // tensor-memory base address
+constexpr uint32_t S_FLAGS = 16;              // [4 items][4] int
+constexpr uint32_t S_META = 80;               // Meta
+constexpr uint32_t S_KQ = 96;                 // per-warp partials of k.q
+constexpr uint32_t S_GKQ = 128;               // float4 per row pair (gk_a, gk_b, gq_a, gq_b)
+constexpr uint32_t S_AK = S_GKQ + 1024;       // float4 per row pair (A_a, A_b, k_a, k_b)
+constexpr uint32_t S_W = S_AK + 1024;         // float per row: w_i (column passes)
+constexpr uint32_t S_IR = S_W + 512;          // float per row: 1 / r16_i
+constexpr uint32_t S_RT = S_IR + 512;         // float per row: row maxima
+constexpr uint32_t S_RD = S_RT + 512;         // uint32 per row: descriptor (processing order)
+constexpr uint32_t S_REDU = S_RD + 512;       // [4 warps][128] partial U
+constexpr uint32_t S_REDP = S_REDU + 2048;    // [4 warps][128] partial P
+constexpr uint32_t S_REDC = S_REDP + 2048;    // [2][4 warps][128] partial column maxima
+constexpr uint32_t S_STAGE = S_REDC + 4096;   // staging buffer, then the head table
+static_assert(S_STAGE % 16 == 0 && S_GKQ % 16 == 0 && S_REDU % 16 == 0, "16-byte aligned");
 
-// A stage: header, k, q, v, (alpha), (row table), head block (offsets within the stage); one
-// or two stages, then the head table.
+// Row descriptor, processing order: original row << 24 | byte offset in the block << 8 | width.
+__device__ __forceinline__ int rd_row(uint32_t d) { return (int)(d >> 24); }
+__device__ __forceinline__ uint32_t rd_off(uint32_t d) { return (d >> 8) & 0xffffu; }
+__device__ __forceinline__ int rd_width(uint32_t d) { return (int)(d & 0xffu); }
+
+// Stage: header, k, q, v, (alpha), (row table), head block.
 struct DPlan {
   uint32_t esz, k_off, q_off, v_off, al_off, rt_off, blk_off, stage, tab, total;
   __host__ __device__ DPlan(int dk, int dv, int io, int gate, int per_row, uint32_t stage_bytes,
-                            int n_heads, int n_stages) {
+                            int n_heads) {
     esz = io == 1 ? 2u : 4u;
     k_off = (uint32_t)sizeof(StageHdr);
     q_off = k_off + dk * esz;
@@ -89,7 +103,7 @@ struct DPlan {
     rt_off = al_off + (gate == 1 ? 4u * dk : 0u);
     blk_off = rt_off + (per_row ? 4u * dk : 0u);  // all offsets multiples of 16
     stage = blk_off + round16(stage_bytes + kSlack);
-    tab = OFF_STAGE + (uint32_t)n_stages * stage;
+    tab = S_STAGE + stage;
     total = tab + round16(20u * (uint32_t)n_heads);
   }
 };
@@ -103,6 +117,7 @@ __device__ __forceinline__ T* sp(uint32_t off) {
 __device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
 __device__ __forceinline__ float2 lo(const float4& v) { return make_float2(v.x, v.y); }
 __device__ __forceinline__ float2 hi(const float4& v) { return make_float2(v.z, v.w); }
+__device__ __forceinline__ float2 dup(float a) { return make_float2(a, a); }
 
 __device__ __forceinline__ float max3abs(float a, float b, float c) {  // max(|a|, |b|, |c|)
   float d;
@@ -114,6 +129,13 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
 }
+// max |.| over the four columns of row a (.x) or row b (.y) of a pair group
+__device__ __forceinline__ float rowmax_x(const float2* v) {
+  return fmaxf(max3abs(v[0].x, v[1].x, v[2].x), fabsf(v[3].x));
+}
+__device__ __forceinline__ float rowmax_y(const float2* v) {
+  return fmaxf(max3abs(v[0].y, v[1].y, v[2].y), fabsf(v[3].y));
+}
 
 __device__ __forceinline__ void cp_async4(void* dst, const void* src) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(dst)), "l"(src)
@@ -122,336 +144,551 @@ __device__ __forceinline__ void cp_async4(void* dst, const void* src) {
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
-// Thread context of one item; FULL = compile-time 128 x 128 tile (every row and lane active).
+// ---- tensor memory, one chunk (16 columns) at a time, loads issued ahead of their use -------
+__device__ __forceinline__ void tm_issue(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+// Wait for every load this thread issued, then hand the registers of `r` over as 8 pairs (the
+// registers are inputs of the same statement as the wait, so nothing reads them earlier).
+__device__ __forceinline__ void tm_take(const uint32_t (&r)[16], float2 (&v)[8]) {
+  uint64_t u[8];
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;\n\t"
+      "mov.b64 %0, {%8,%9};\n\tmov.b64 %1, {%10,%11};\n\tmov.b64 %2, {%12,%13};\n\t"
+      "mov.b64 %3, {%14,%15};\n\tmov.b64 %4, {%16,%17};\n\tmov.b64 %5, {%18,%19};\n\t"
+      "mov.b64 %6, {%20,%21};\n\tmov.b64 %7, {%22,%23};"
+      : "=l"(u[0]), "=l"(u[1]), "=l"(u[2]), "=l"(u[3]), "=l"(u[4]), "=l"(u[5]), "=l"(u[6]),
+        "=l"(u[7])
+      : "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15])
+      : "memory");
+#pragma unroll
+  for (int e = 0; e < 8; ++e) v[e] = *reinterpret_cast<const float2*>(&u[e]);
+}
+
+// Run body(ch, v) over chunks 0..nch-1 (nch even) of the thread's tile, each chunk's load in
+// flight while the previous chunk is processed.
+template <class F>
+__device__ __forceinline__ void sweep(uint32_t tm, int nch, F&& body) {
+  uint32_t ra[16], rb[16];
+  if (nch <= 0) return;
+  tm_issue(tm, ra);
+#pragma unroll 1
+  for (int ch = 0; ch < nch; ch += 2) {
+    float2 v[8];
+    tm_take(ra, v);
+    tm_issue(tm + 16u * (ch + 1), rb);
+    body(ch, v);
+    float2 w[8];
+    tm_take(rb, w);
+    if (ch + 2 < nch) tm_issue(tm + 16u * (ch + 2), ra);
+    body(ch + 1, w);
+  }
+}
+
+// ---- unpack: the lane's four columns of two rows (a, b) as pairs (a_e, b_e) of exact codes --
+__device__ __forceinline__ float2 f2u(uint32_t x, uint32_t y) {
+  return make_float2(__uint_as_float(x), __uint_as_float(y));
+}
+
+template <int B>
+__device__ __forceinline__ void unpack_pair(const uint8_t* ra, const uint8_t* rb, int lane,
+                                            float2 (&x)[4]);
+
+template <>
+__device__ __forceinline__ void unpack_pair<2>(const uint8_t* ra, const uint8_t* rb, int lane,
+                                               float2 (&x)[4]) {
+  const uint32_t va = ra[lane], vb = rb[lane];  // f = 2^23 + u 4^e ; code = f 4^-e - (2^(23-2e) + 2)
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const uint32_t m = 3u << (2 * e);
+    x[e] = __ffma2_rn(f2u(kMagicBits | (va & m), kMagicBits | (vb & m)),
+                      dup(1.0f / float(1u << (2 * e))), dup(-(float(1u << (23 - 2 * e)) + 2.0f)));
+  }
+}
+
+template <>
+__device__ __forceinline__ void unpack_pair<4>(const uint8_t* ra, const uint8_t* rb, int lane,
+                                               float2 (&x)[4]) {
+  const uint32_t va = reinterpret_cast<const uint16_t*>(ra)[lane];
+  const uint32_t vb = reinterpret_cast<const uint16_t*>(rb)[lane];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const uint32_t m = 15u << (4 * e);
+    x[e] = __ffma2_rn(f2u(kMagicBits | (va & m), kMagicBits | (vb & m)),
+                      dup(1.0f / float(1u << (4 * e))), dup(-(float(1u << (23 - 4 * e)) + 8.0f)));
+  }
+}
+
+__device__ __forceinline__ uint32_t bits24(const uint8_t* row, int lane) {  // 6-bit: lane's 24 bits
+  const int byte = 3 * lane;
+  const uint32_t* w = reinterpret_cast<const uint32_t*>(row + (byte & ~3));
+  return __funnelshift_r(w[0], w[1], (byte & 3) * 8);
+}
+
+template <>
+__device__ __forceinline__ void unpack_pair<6>(const uint8_t* ra, const uint8_t* rb, int lane,
+                                               float2 (&x)[4]) {
+  const uint32_t va = bits24(ra, lane), vb = bits24(rb, lane);
+  const uint32_t ha = va >> 12, hb = vb >> 12;
+  const float2 s1 = dup(1.0f / 64.0f);
+  const float2 o0 = dup(-(8388608.f + 32.f)), o1 = dup(-(131072.f + 32.f));
+  x[0] = __fadd2_rn(f2u(kMagicBits | (va & 63u), kMagicBits | (vb & 63u)), o0);
+  x[1] = __ffma2_rn(f2u(kMagicBits | (va & (63u << 6)), kMagicBits | (vb & (63u << 6))), s1, o1);
+  x[2] = __fadd2_rn(f2u(kMagicBits | (ha & 63u), kMagicBits | (hb & 63u)), o0);
+  x[3] = __ffma2_rn(f2u(kMagicBits | (ha & (63u << 6)), kMagicBits | (hb & (63u << 6))), s1, o1);
+}
+
+template <>
+__device__ __forceinline__ void unpack_pair<8>(const uint8_t* ra, const uint8_t* rb, int lane,
+                                               float2 (&x)[4]) {
+  const uint32_t va = reinterpret_cast<const uint32_t*>(ra)[lane];
+  const uint32_t vb = reinterpret_cast<const uint32_t*>(rb)[lane];
+  const float2 m = dup(-(kMagic + 128.f));
+#pragma unroll
+  for (int e = 0; e < 4; ++e)
+    x[e] = __fadd2_rn(f2u(__byte_perm(va, kMagicBits, 0x7540u + e),
+                          __byte_perm(vb, kMagicBits, 0x7540u + e)), m);
+}
+
+template <>
+__device__ __forceinline__ void unpack_pair<16>(const uint8_t* ra, const uint8_t* rb, int lane,
+                                                float2 (&x)[4]) {
+  // fp16 rows start on 4-byte boundaries: two 32-bit loads per row
+  const uint32_t* wa = reinterpret_cast<const uint32_t*>(ra) + 2 * lane;
+  const uint32_t* wb = reinterpret_cast<const uint32_t*>(rb) + 2 * lane;
+  const uint32_t a0 = wa[0], a1 = wa[1], b0 = wb[0], b1 = wb[1];
+  const __half2 ha0 = *reinterpret_cast<const __half2*>(&a0), ha1 = *reinterpret_cast<const __half2*>(&a1);
+  const __half2 hb0 = *reinterpret_cast<const __half2*>(&b0), hb1 = *reinterpret_cast<const __half2*>(&b1);
+  x[0] = f2(__low2float(ha0), __low2float(hb0));
+  x[1] = f2(__high2float(ha0), __high2float(hb0));
+  x[2] = f2(__low2float(ha1), __low2float(hb1));
+  x[3] = f2(__high2float(ha1), __high2float(hb1));
+}
+
+// Either row of a pair with its own width (key-row units, rows of two widths).
+__device__ __forceinline__ void unpack_mixed(int wa, const uint8_t* ra, int wb, const uint8_t* rb,
+                                             int lane, float2 (&x)[4]) {
+  float xa[4], xb[4];
+  unpack4_rt(wa, ra, lane, xa);
+  unpack4_rt(wb, rb, lane, xb);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) x[e] = f2(xa[e], xb[e]);
+}
+
+template <int B>
+__device__ __forceinline__ constexpr uint32_t row_bytes_of(int dv) {
+  return (uint32_t)dv * B / 8;
+}
+
+// Thread context of one item; FULL = compile-time 128 x 128 tile.
 template <bool FULL>
 struct Ctx {
-  int tid, warp, lane, dk_, dv_;
-  bool act_;   // the lane's columns are < d_v
-  bool wact_;  // the warp's rows are < d_k (d_k is a multiple of 16)
+  int tid, warp, lane, dk_, dv_, nch_;
+  bool act_;  // the lane's columns are < d_v
+  uint32_t tm;
+  int* flags;
   __device__ int dk() const { return FULL ? kMaxD : dk_; }
   __device__ int dv() const { return FULL ? kMaxD : dv_; }
   __device__ bool act() const { return FULL || act_; }
-  __device__ bool wact() const { return FULL || wact_; }
-  const uint8_t* blk;
-  int* flags;  // the item's flag words
-  uint32_t tm;  // tensor-memory address of the thread's 64 values
-  __device__ float4* rowG() const { return sp<float4>(OFF_ROWG); }
-  __device__ float4* rowU() const { return sp<float4>(OFF_ROWU); }
-  __device__ float2* rowW2() const { return sp<float2>(OFF_ROWW2); }
-  __device__ float2* rowIR2() const { return sp<float2>(OFF_ROWIR2); }
-  __device__ uint32_t* rowtab() const { return sp<uint32_t>(OFF_ROWTAB); }
-  __device__ float* rowtmp() const { return sp<float>(OFF_ROWTMP) + warp * kRows; }
-  __device__ int row0() const { return warp * kRows; }
+  __device__ int nch() const { return FULL ? kMaxCh : nch_; }  // chunks of the warp's rows
+  __device__ int row0() const { return warp * kRW; }
 };
 
-// Row geometry of a head block: fixed width (head units, fp16 heads) or the row table.
-template <int MODE>
-struct Geo {
-  uint32_t base, rb;
-  template <bool FULL>
-  __device__ Geo(const Ctx<FULL>& c)
-      : base(MODE == MODE_PIVOT ? 0u : 2u * (c.dk() + c.dv())), rb((uint32_t)c.dv() * MODE / 8) {}
-  __device__ uint32_t off(int i) const { return base + (uint32_t)i * rb; }
-  __device__ int width(int) const { return MODE; }
-};
-template <>
-struct Geo<MODE_ROWS> {
-  const uint32_t* tab;
-  template <bool FULL>
-  __device__ Geo(const Ctx<FULL>& c) : tab(c.rowtab()) {}
-  __device__ uint32_t off(int i) const { return row_off(tab[i]); }
-  __device__ int width(int i) const { return row_width(tab[i]); }
-};
-
-// Sum / max over the 8 warps of the partials in red[w * stride + 4 lane .. +3].
-__device__ __forceinline__ float4 sum8(const float* red, int stride, int lane) {
-  float2 a = f2(0.f, 0.f), b = a;
+// ---- pass A: exact codes into tensor memory, partial U and P ------------------------------
+// Head units of width B (16: fp16 head): rows in key order, row p at base + p * rb.
+template <int B, bool FULL>
+__device__ __forceinline__ void pass_a_head(const Ctx<FULL>& c, const uint8_t* blk) {
+  const int dv = c.dv();
+  const uint32_t rb = row_bytes_of<B>(dv);
+  const uint8_t* row0 = blk + (B == 16 ? 0u : 2u * (c.dk() + dv)) + (uint32_t)c.row0() * rb;
+  const float4* gkq = sp<float4>(S_GKQ) + c.row0() / 2;
+  float2 U[4], P[4];
 #pragma unroll
-  for (int w = 0; w < kWarps; ++w) {
-    const float4 v = *reinterpret_cast<const float4*>(red + w * stride + 4 * lane);
-    a = __fadd2_rn(a, lo(v));
-    b = __fadd2_rn(b, hi(v));
-  }
-  return make_float4(a.x, a.y, b.x, b.y);
-}
-
-__device__ __forceinline__ float4 max8(const float* red, int lane) {
-  float4 m = *reinterpret_cast<const float4*>(red + 4 * lane);
+  for (int e = 0; e < 4; ++e) U[e] = P[e] = f2(0.f, 0.f);
+#pragma unroll 2
+  for (int ch = 0; ch < c.nch(); ++ch) {
+    float2 v[8];
 #pragma unroll
-  for (int w = 1; w < kWarps; w += 2) {
-    const float4 a = *reinterpret_cast<const float4*>(red + w * kMaxD + 4 * lane);
-    const float4 b =
-        *reinterpret_cast<const float4*>(red + (w + 1 < kWarps ? w + 1 : w) * kMaxD + 4 * lane);
-    m.x = max3(m.x, a.x, b.x);
-    m.y = max3(m.y, a.y, b.y);
-    m.z = max3(m.z, a.z, b.z);
-    m.w = max3(m.w, a.w, b.w);
-  }
-  return make_float4(fmaxf(m.x, kScaleFloor), fmaxf(m.y, kScaleFloor), fmaxf(m.z, kScaleFloor),
-                     fmaxf(m.w, kScaleFloor));
-}
-
-// ---- pass A: exact codes into tensor memory, partial dot products -------------------------
-template <int MODE, bool FULL>
-__device__ __forceinline__ void pass_a(const Ctx<FULL>& c) {
-  const Geo<MODE> geo(c);
-  // two accumulator sets (even / odd rows) halve the dependent-add chains
-  float2 U0 = f2(0.f, 0.f), U1 = U0, P0 = U0, P1 = U0, U2 = U0, U3 = U0, P2 = U0, P3 = U0;
-  if (c.wact()) {
-    float4 icv = make_float4(1.f, 1.f, 1.f, 1.f);
-    if (MODE == MODE_ROWS && c.act()) {  // 1/c16 of the lane's columns, for fp16 rows
-      const uint2 ch = reinterpret_cast<const uint2*>(c.blk + 2 * c.dk())[c.lane];
-      const float2 a01 = __half22float2(*reinterpret_cast<const __half2*>(&ch.x));
-      const float2 a23 = __half22float2(*reinterpret_cast<const __half2*>(&ch.y));
-      icv = make_float4(rcp_f16val(a01.x), rcp_f16val(a01.y), rcp_f16val(a23.x), rcp_f16val(a23.y));
-    }
-#pragma unroll 1
-    for (int ch = 0; ch < kChunks; ++ch) {
-      float2 v[8];
+    for (int pr = 0; pr < 2; ++pr) {
+      const uint8_t* ra = row0 + (uint32_t)(4 * ch + 2 * pr) * rb;
+      float2 x[4];
+      if (c.act()) {
+        unpack_pair<B>(ra, ra + rb, c.lane, x);
+      } else {
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int i = c.row0() + 4 * ch + r;
-        float2 x01 = f2(0.f, 0.f), x23 = x01;
-        const int b = geo.width(i);
-        if (c.act()) {
-          const uint8_t* row = c.blk + geo.off(i);
-          if constexpr (MODE == MODE_ROWS)
-            unpack4x2_rt(b, row, c.lane, x01, x23);
-          else
-            unpack4x2<MODE>(row, c.lane, x01, x23);
-        }
-        if (MODE == MODE_ROWS && b == 16) {  // fp16 row inside a scaled head: x = value / c_j
-          x01 = __fmul2_rn(x01, lo(icv));
-          x23 = __fmul2_rn(x23, hi(icv));
-        }
-        v[2 * r] = x01;
-        v[2 * r + 1] = x23;
-        const float4 g = c.rowG()[i];  // (gk, gk, gq, gq)
-        if (r & 1) {
-          U2 = __ffma2_rn(x01, lo(g), U2);
-          U3 = __ffma2_rn(x23, lo(g), U3);
-          P2 = __ffma2_rn(x01, hi(g), P2);
-          P3 = __ffma2_rn(x23, hi(g), P3);
-        } else {
-          U0 = __ffma2_rn(x01, lo(g), U0);
-          U1 = __ffma2_rn(x23, lo(g), U1);
-          P0 = __ffma2_rn(x01, hi(g), P0);
-          P1 = __ffma2_rn(x23, hi(g), P1);
-        }
+        for (int e = 0; e < 4; ++e) x[e] = f2(0.f, 0.f);
       }
-      tmem_st16x2(c.tm + 16 * ch, v);
+      const float4 g = gkq[2 * ch + pr];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        U[e] = __ffma2_rn(x[e], lo(g), U[e]);
+        P[e] = __ffma2_rn(x[e], hi(g), P[e]);
+        v[4 * pr + e] = x[e];
+      }
     }
+    tmem_st16x2(c.tm + 16u * ch, v);
   }
-  U0 = __fadd2_rn(U0, U2);
-  U1 = __fadd2_rn(U1, U3);
-  P0 = __fadd2_rn(P0, P2);
-  P1 = __fadd2_rn(P1, P3);
-  float* red = sp<float>(OFF_REDA) + c.warp * 2 * kMaxD + 4 * c.lane;
-  *reinterpret_cast<float4*>(red) = make_float4(U0.x, U0.y, U1.x, U1.y);
-  *reinterpret_cast<float4*>(red + kMaxD) = make_float4(P0.x, P0.y, P1.x, P1.y);
+  *reinterpret_cast<float4*>(sp<float>(S_REDU) + c.warp * kMaxD + 4 * c.lane) =
+      make_float4(U[0].x + U[0].y, U[1].x + U[1].y, U[2].x + U[2].y, U[3].x + U[3].y);
+  *reinterpret_cast<float4*>(sp<float>(S_REDP) + c.warp * kMaxD + 4 * c.lane) =
+      make_float4(P[0].x + P[0].y, P[1].x + P[1].y, P[2].x + P[2].y, P[3].x + P[3].y);
 }
 
-// ---- pass B: M_new = x (A_i c_j) + k_i b_j, row maxima of |M_new| -------------------------
-// check16: 0 no fp16 rows, 1 every row is fp16 (fp16 head), 2 per the row table.
+// Key-row units: per-chunk width dispatch (rows are width-sorted), fp16 rows scaled by 1/c_j.
 template <bool FULL>
-__device__ __forceinline__ void pass_b(const Ctx<FULL>& c, const float4& cv, const float4& bv,
-                                       float* s_new, int check16, bool fit) {
-  bool of = false;
-  if (c.wact()) {
+__device__ __forceinline__ void pass_a_rows(const Ctx<FULL>& c, const uint8_t* blk, const float4& icv) {
+  const float4* gkq = sp<float4>(S_GKQ) + c.row0() / 2;
+  const uint4* rd4 = reinterpret_cast<const uint4*>(sp<uint32_t>(S_RD) + c.row0());
+  float2 U[4], P[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) U[e] = P[e] = f2(0.f, 0.f);
+  const float ic[4] = {icv.x, icv.y, icv.z, icv.w};
 #pragma unroll 1
-    for (int ch = 0; ch < kChunks; ++ch) {
-      float2 v[8];
-      tmem_ld16x2(c.tm + 16 * ch, v);
-      float rm[4];
+  for (int ch = 0; ch < c.nch(); ++ch) {
+    const uint4 d = rd4[ch];
+    const uint32_t ds[4] = {d.x, d.y, d.z, d.w};
+    float2 v[8];
+#pragma unroll
+    for (int pr = 0; pr < 2; ++pr) {
+      const uint32_t da = ds[2 * pr], db = ds[2 * pr + 1];
+      const int wa = rd_width(da), wb = rd_width(db);
+      const uint8_t* ra = blk + rd_off(da);
+      const uint8_t* rbp = blk + rd_off(db);
+      float2 x[4];
+      if (!c.act()) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) x[e] = f2(0.f, 0.f);
+      } else if (wa == wb) {
+        switch (wa) {
+          case 2: unpack_pair<2>(ra, rbp, c.lane, x); break;
+          case 4: unpack_pair<4>(ra, rbp, c.lane, x); break;
+          case 6: unpack_pair<6>(ra, rbp, c.lane, x); break;
+          case 8: unpack_pair<8>(ra, rbp, c.lane, x); break;
+          default: unpack_pair<16>(ra, rbp, c.lane, x); break;
+        }
+      } else {
+        unpack_mixed(wa, ra, wb, rbp, c.lane, x);
+      }
+      if (wa == 16 || wb == 16) {  // fp16 rows hold values: x = value / c_j
+#pragma unroll
+        for (int e = 0; e < 4; ++e) x[e] = f2(wa == 16 ? x[e].x * ic[e] : x[e].x, wb == 16 ? x[e].y * ic[e] : x[e].y);
+      }
+      const float4 g = gkq[2 * ch + pr];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        U[e] = __ffma2_rn(x[e], lo(g), U[e]);
+        P[e] = __ffma2_rn(x[e], hi(g), P[e]);
+        v[4 * pr + e] = x[e];
+      }
+    }
+    tmem_st16x2(c.tm + 16u * ch, v);
+  }
+  *reinterpret_cast<float4*>(sp<float>(S_REDU) + c.warp * kMaxD + 4 * c.lane) =
+      make_float4(U[0].x + U[0].y, U[1].x + U[1].y, U[2].x + U[2].y, U[3].x + U[3].y);
+  *reinterpret_cast<float4*>(sp<float>(S_REDP) + c.warp * kMaxD + 4 * c.lane) =
+      make_float4(P[0].x + P[0].y, P[1].x + P[1].y, P[2].x + P[2].y, P[3].x + P[3].y);
+}
+
+// ---- pass B: M_new = x (A_i c_j) + k_i b_j in place, row maxima into S_RT -------------------
+// KIND 0: quantized head (row maxima); 1: fp16 head (fp16 range check, no maxima); 2: key-row
+// units (row maxima; range check of the fp16 rows).
+template <int KIND, bool WS, bool FULL>
+__device__ __forceinline__ void pass_b(const Ctx<FULL>& c, const float4& cv, const float4& bv,
+                                       float* s_new) {
+  const float2 cc[4] = {dup(cv.x), dup(cv.y), dup(cv.z), dup(cv.w)};
+  const float2 bb[4] = {dup(bv.x), dup(bv.y), dup(bv.z), dup(bv.w)};
+  const float4* ak = sp<float4>(S_AK) + c.row0() / 2;
+  float4* rt = reinterpret_cast<float4*>(sp<float>(S_RT) + c.row0());
+  const uint4* rd4 = reinterpret_cast<const uint4*>(sp<uint32_t>(S_RD) + c.row0());
+  const int dv = c.dv();
+  bool of = false;
+  sweep(c.tm, c.nch(), [&](int ch, float2 (&v)[8]) {
+    float rm[4];
+#pragma unroll
+    for (int pr = 0; pr < 2; ++pr) {
+      const float4 f = ak[2 * ch + pr];
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        v[4 * pr + e] = __ffma2_rn(v[4 * pr + e], __fmul2_rn(lo(f), cc[e]), __fmul2_rn(hi(f), bb[e]));
+      if (KIND != 1) {
+        rm[2 * pr] = warp_max_nonneg(rowmax_x(v + 4 * pr));
+        rm[2 * pr + 1] = warp_max_nonneg(rowmax_y(v + 4 * pr));
+      }
+    }
+    if (KIND == 1) {
+      float m = 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) m = max3abs(m, v[e].x, v[e].y);
+      of |= !(m < 65520.f);
+    }
+    if (KIND != 1 && c.lane == 0) rt[ch] = make_float4(rm[0], rm[1], rm[2], rm[3]);
+    if (KIND == 2 || WS) {
+      const uint4 d = rd4[ch];
+      const uint32_t ds[4] = {d.x, d.y, d.z, d.w};
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
-        const int i = c.row0() + 4 * ch + r;
-        const float4 u = c.rowU()[i];  // (A, A, k, k)
-        const float2 s0 = __ffma2_rn(v[2 * r], __fmul2_rn(lo(u), lo(cv)), __fmul2_rn(hi(u), lo(bv)));
-        const float2 s1 = __ffma2_rn(v[2 * r + 1], __fmul2_rn(lo(u), hi(cv)), __fmul2_rn(hi(u), hi(bv)));
-        v[2 * r] = s0;
-        v[2 * r + 1] = s1;
-        if (fit) rm[r] = warp_max_nonneg(fmaxf(max3abs(s0.x, s0.y, s1.x), fabsf(s1.y)));
-        if (check16 == 1 || (check16 == 2 && row_width(c.rowtab()[i]) == 16))  // RN16 -> inf
-          if (c.act()) of |= !(fmaxf(max3abs(s0.x, s0.y, s1.x), fabsf(s1.y)) < 65520.f);
-        if (s_new != nullptr && c.act())
-          *reinterpret_cast<float4*>(s_new + (size_t)i * c.dv() + 4 * c.lane) =
-              make_float4(s0.x, s0.y, s1.x, s1.y);
+        const float2* g = v + 4 * (r >> 1);
+        const float4 row = (r & 1) ? make_float4(g[0].y, g[1].y, g[2].y, g[3].y)
+                                   : make_float4(g[0].x, g[1].x, g[2].x, g[3].x);
+        if (KIND == 2 && rd_width(ds[r]) == 16 && c.act())
+          of |= !(fmaxf(max3abs(row.x, row.y, row.z), fabsf(row.w)) < 65520.f);
+        if (WS && c.act())
+          *reinterpret_cast<float4*>(s_new + (size_t)rd_row(ds[r]) * dv + 4 * c.lane) = row;
       }
-      tmem_st16x2(c.tm + 16 * ch, v);
-      if (fit && c.lane == 0)
-        *reinterpret_cast<float4*>(c.rowtmp() + 4 * ch) = make_float4(rm[0], rm[1], rm[2], rm[3]);
     }
-  }
+    tmem_st16x2(c.tm + 16u * ch, v);
+  });
   if (of) atomicOr(&c.flags[F_RANGE], 1);
   tmem_wait_st();
   __syncwarp();
 }
 
-// Row scales from the row maxima in rowtmp: r_i = max(m_i / Q_i, 2^-14), w_i = 1 / (r_i Q_i);
-// fp16 rows get r = w = 0. Lane s < 16 returns r of row 16w + s.
+// Row scales from the row maxima in S_RT, one row per lane: r = max(m / Q, 2^-14) (at most the
+// largest fp16), w = 1 / (r Q) into S_W; fp16 rows get r = w = 0. Returns the lane's r.
 template <bool FULL>
-__device__ __forceinline__ float row_scales(const Ctx<FULL>& c, int mode, bool check) {
-  float r = 0.f;
-  if (c.lane < kRows) {
-    const int i = c.row0() + c.lane;
-    float w = 0.f;
-    if (c.wact()) {
-      const int b = mode == MODE_ROWS ? row_width(c.rowtab()[i]) : mode;
-      if (b != 16) {
-        const float Q = (float)q_of_width(b);
-        const float inv_q = b == 2 ? 1.0f : b == 4 ? 1.0f / 7.0f : b == 6 ? 1.0f / 31.0f : 1.0f / 127.0f;
-        const float rq = div_q(c.rowtmp()[c.lane], Q, inv_q);  // exactly m / Q
-        if (check && !(rq < 65520.f)) atomicOr(&c.flags[F_RANGE], 1);
-        r = fminf(fmaxf(rq, kScaleFloor), 65504.f);  // 65504: the largest finite fp16 value
-        w = rcp_approx(__fmul_rn(r, Q));
-      }
+__device__ __forceinline__ float row_scales(const Ctx<FULL>& c, bool check) {
+  const int p = c.row0() + c.lane;
+  float r = 0.f, w = 0.f;
+  if (p < c.dk()) {
+    const int b = rd_width(sp<uint32_t>(S_RD)[p]);
+    if (b != 16) {
+      const float Q = (float)q_of_width(b);
+      const float inv_q = b == 2 ? 1.0f : b == 4 ? 1.0f / 7.0f : b == 6 ? 1.0f / 31.0f : 1.0f / 127.0f;
+      const float rq = div_q(sp<float>(S_RT)[p], Q, inv_q);  // exactly m / Q
+      if (check && !(rq < 65520.f)) atomicOr(&c.flags[F_RANGE], 1);
+      r = fminf(fmaxf(rq, kScaleFloor), 65504.f);
+      w = rcp_approx(__fmul_rn(r, Q));
     }
-    c.rowW2()[i] = f2(w, w);
   }
+  sp<float>(S_W)[p] = w;
   __syncwarp();
   return r;
 }
 
-// Column pass: max_i |S_ij| w_i over the warp's rows, into red[warp].
+// Column pass: max_i |S_ij| w_i over the warp's rows into red[warp].
 template <bool FULL>
 __device__ __forceinline__ void col_pass(const Ctx<FULL>& c, float* red) {
-  float cm0 = 0.f, cm1 = 0.f, cm2 = 0.f, cm3 = 0.f, cn0 = 0.f, cn1 = 0.f, cn2 = 0.f, cn3 = 0.f;
-  if (c.wact()) {
-    const float4* w2 = reinterpret_cast<const float4*>(c.rowW2() + c.row0());
-#pragma unroll 1
-    for (int ch = 0; ch < kChunks; ++ch) {
-      float2 v[8];
-      tmem_ld16x2(c.tm + 16 * ch, v);
+  const float2* w2 = reinterpret_cast<const float2*>(sp<float>(S_W) + c.row0());
+  float m0[4] = {0.f, 0.f, 0.f, 0.f}, m1[4] = {0.f, 0.f, 0.f, 0.f};
+  sweep(c.tm, c.nch(), [&](int ch, float2 (&v)[8]) {
+    const float2 wa = w2[2 * ch], wb = w2[2 * ch + 1];
 #pragma unroll
-      for (int r = 0; r < 4; r += 2) {
-        const float4 ww = w2[2 * ch + r / 2];  // (w_s, w_s, w_s+1, w_s+1)
-        const float2 a0 = __fmul2_rn(v[2 * r], lo(ww));
-        const float2 a1 = __fmul2_rn(v[2 * r + 1], lo(ww));
-        const float2 b0 = __fmul2_rn(v[2 * r + 2], hi(ww));
-        const float2 b1 = __fmul2_rn(v[2 * r + 3], hi(ww));
-        if (r == 0) {
-          cm0 = max3abs(cm0, a0.x, b0.x);
-          cm1 = max3abs(cm1, a0.y, b0.y);
-          cm2 = max3abs(cm2, a1.x, b1.x);
-          cm3 = max3abs(cm3, a1.y, b1.y);
-        } else {
-          cn0 = max3abs(cn0, a0.x, b0.x);
-          cn1 = max3abs(cn1, a0.y, b0.y);
-          cn2 = max3abs(cn2, a1.x, b1.x);
-          cn3 = max3abs(cn3, a1.y, b1.y);
-        }
-      }
+    for (int e = 0; e < 4; ++e) {
+      const float2 p = __fmul2_rn(v[e], wa);
+      const float2 q = __fmul2_rn(v[4 + e], wb);
+      m0[e] = max3abs(m0[e], p.x, p.y);
+      m1[e] = max3abs(m1[e], q.x, q.y);
     }
-  }
+  });
   *reinterpret_cast<float4*>(red + c.warp * kMaxD + 4 * c.lane) =
-      make_float4(fmaxf(cm0, cn0), fmaxf(cm1, cn1), fmaxf(cm2, cn2), fmaxf(cm3, cn3));
+      make_float4(fmaxf(m0[0], m1[0]), fmaxf(m0[1], m1[1]), fmaxf(m0[2], m1[2]), fmaxf(m0[3], m1[3]));
 }
 
-// Row pass of a later alternation: row maxima of |S_ij| v_j into rowtmp.
+// Row pass of a later alternation: row maxima of |S_ij| v_j into S_RT.
 template <bool FULL>
 __device__ __forceinline__ void row_pass(const Ctx<FULL>& c, const float4& icv) {
-  if (c.wact()) {
-#pragma unroll 1
-    for (int ch = 0; ch < kChunks; ++ch) {
-      float2 v[8];
-      tmem_ld16x2(c.tm + 16 * ch, v);
-      float rm[4];
+  const float2 ic[4] = {dup(icv.x), dup(icv.y), dup(icv.z), dup(icv.w)};
+  float4* rt = reinterpret_cast<float4*>(sp<float>(S_RT) + c.row0());
+  sweep(c.tm, c.nch(), [&](int ch, float2 (&v)[8]) {
+    float rm[4];
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const float2 p = __fmul2_rn(v[2 * r], lo(icv));
-        const float2 q = __fmul2_rn(v[2 * r + 1], hi(icv));
-        rm[r] = warp_max_nonneg(fmaxf(max3abs(p.x, p.y, q.x), fabsf(q.y)));
-      }
-      if (c.lane == 0)
-        *reinterpret_cast<float4*>(c.rowtmp() + 4 * ch) = make_float4(rm[0], rm[1], rm[2], rm[3]);
+    for (int pr = 0; pr < 2; ++pr) {
+      float2 p[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) p[e] = __fmul2_rn(v[4 * pr + e], ic[e]);
+      rm[2 * pr] = warp_max_nonneg(rowmax_x(p));
+      rm[2 * pr + 1] = warp_max_nonneg(rowmax_y(p));
     }
-  }
+    if (c.lane == 0) rt[ch] = make_float4(rm[0], rm[1], rm[2], rm[3]);
+  });
   __syncwarp();
 }
 
-// ---- requantize, pack and store the scaled head ---------------------------------------------
-template <int MODE, bool FULL>
-__device__ __forceinline__ void requant(const Ctx<FULL>& c, uint8_t* dst, const float4& cm, float r) {
-  const Geo<MODE> geo(c);
-  const __half2 c01 = __floats2half2_rn(cm.x, cm.y), c23 = __floats2half2_rn(cm.z, cm.w);
-  const float2 fc01 = __half22float2(c01), fc23 = __half22float2(c23);
-  const float2 ic01 = f2(rcp_f16val(fc01.x), rcp_f16val(fc01.y));  // correctly rounded
-  const float2 ic23 = f2(rcp_f16val(fc23.x), rcp_f16val(fc23.y));
-  __half* r16s = reinterpret_cast<__half*>(c.rowtmp());
-  if (c.lane < kRows) {
-    const __half r16 = __float2half_rn(r);
-    const float ir = r > 0.f ? rcp_f16val(__half2float(r16)) : 0.f;
-    c.rowIR2()[c.row0() + c.lane] = f2(ir, ir);
-    r16s[c.lane] = r16;
+// Max over the four warps' partial column maxima of the lane's columns, floored at 2^-14.
+__device__ __forceinline__ float4 max4(const float* red, int lane) {
+  const float4 a = *reinterpret_cast<const float4*>(red + 4 * lane);
+  const float4 b = *reinterpret_cast<const float4*>(red + kMaxD + 4 * lane);
+  const float4 c = *reinterpret_cast<const float4*>(red + 2 * kMaxD + 4 * lane);
+  const float4 d = *reinterpret_cast<const float4*>(red + 3 * kMaxD + 4 * lane);
+  return make_float4(max3(fmaxf(a.x, b.x), c.x, fmaxf(d.x, kScaleFloor)),
+                     max3(fmaxf(a.y, b.y), c.y, fmaxf(d.y, kScaleFloor)),
+                     max3(fmaxf(a.z, b.z), c.z, fmaxf(d.z, kScaleFloor)),
+                     max3(fmaxf(a.w, b.w), c.w, fmaxf(d.w, kScaleFloor)));
+}
+
+__device__ __forceinline__ float4 sum4(const float* red, int lane) {
+  const float4 a = *reinterpret_cast<const float4*>(red + 4 * lane);
+  const float4 b = *reinterpret_cast<const float4*>(red + kMaxD + 4 * lane);
+  const float4 c = *reinterpret_cast<const float4*>(red + 2 * kMaxD + 4 * lane);
+  const float4 d = *reinterpret_cast<const float4*>(red + 3 * kMaxD + 4 * lane);
+  const float2 x = __fadd2_rn(__fadd2_rn(lo(a), lo(b)), __fadd2_rn(lo(c), lo(d)));
+  const float2 y = __fadd2_rn(__fadd2_rn(hi(a), hi(b)), __fadd2_rn(hi(c), hi(d)));
+  return make_float4(x.x, x.y, y.x, y.y);
+}
+
+// ---- requantize, pack and store ----------------------------------------------------------
+// Row scales: r16_i to the block (at the original row), 1/r16_i into S_IR; column scales: c16.
+// Returns the lane's correctly rounded 1/c16 of its four columns.
+template <bool FULL>
+__device__ __forceinline__ float4 store_scales(const Ctx<FULL>& c, uint8_t* dst, const float4& cm, float r) {
+  const int p = c.row0() + c.lane;
+  if (p < c.dk()) {
+    const uint32_t d = sp<uint32_t>(S_RD)[p];
+    const bool q = rd_width(d) != 16;
+    const __half r16 = __float2half_rn(q ? r : 0.f);
+    sp<float>(S_IR)[p] = q ? rcp_f16val(__half2float(r16)) : 0.f;
+    reinterpret_cast<__half*>(dst)[rd_row(d)] = r16;
   }
-  __syncwarp();
-  if (c.wact() && c.lane < 2)
-    reinterpret_cast<uint4*>(dst)[2 * c.warp + c.lane] = reinterpret_cast<const uint4*>(r16s)[c.lane];
+  const __half2 c01 = __floats2half2_rn(cm.x, cm.y), c23 = __floats2half2_rn(cm.z, cm.w);
   if (c.warp == 0 && c.act()) {
     uint2 cc;
     cc.x = *reinterpret_cast<const uint32_t*>(&c01);
     cc.y = *reinterpret_cast<const uint32_t*>(&c23);
     reinterpret_cast<uint2*>(dst + 2 * c.dk())[c.lane] = cc;
   }
-  if (!c.wact()) return;
-#pragma unroll 1
-  for (int ch = 0; ch < kChunks; ++ch) {
-    float2 v[8];
-    tmem_ld16x2(c.tm + 16 * ch, v);
+  __syncwarp();
+  const float2 f01 = __half22float2(c01), f23 = __half22float2(c23);
+  return make_float4(rcp_f16val(f01.x), rcp_f16val(f01.y), rcp_f16val(f23.x), rcp_f16val(f23.y));
+}
+
+// Codes of one pair group (rows a, b of a chunk): y = fl(S fl(1/r16)) * fl(1/c16) + magic.
+__device__ __forceinline__ void quant_pair(const float2* v, float2 ir, const float2 (&ic)[4],
+                                           float mgv, float ya[4], float yb[4]) {
+  const float2 mg = dup(mgv);
 #pragma unroll
-    for (int r2 = 0; r2 < 4; ++r2) {
-      const int i = c.row0() + 4 * ch + r2;
-      uint8_t* row = dst + geo.off(i);
-      const int b = geo.width(i);
-      if (MODE == MODE_ROWS && b == 16) {
-        store4_f16x2(row, c.lane, v[2 * r2], v[2 * r2 + 1], c.act());
-      } else {
-        const float2 ir = c.rowIR2()[i];
-        const float mgv = kMagic + (float)(1 << (b - 1));
-        const float2 mg = f2(mgv, mgv);
-        const float2 y0 = __ffma2_rn(__fmul2_rn(v[2 * r2], ir), ic01, mg);
-        const float2 y1 = __ffma2_rn(__fmul2_rn(v[2 * r2 + 1], ir), ic23, mg);
-        const float y[4] = {y0.x, y0.y, y1.x, y1.y};
-        if constexpr (MODE == MODE_ROWS) {
-          switch (b) {
-            case 2: store4<2>(row, c.lane, y, c.act()); break;
-            case 4: store4<4>(row, c.lane, y, c.act()); break;
-            case 6: store4<6>(row, c.lane, y, c.act()); break;
-            default: store4<8>(row, c.lane, y, c.act()); break;
-          }
-        } else {
-          store4<MODE>(row, c.lane, y, c.act());
-        }
-      }
-    }
+  for (int e = 0; e < 4; ++e) {
+    const float2 y = __ffma2_rn(__fmul2_rn(v[e], ir), ic[e], mg);
+    ya[e] = y.x;
+    yb[e] = y.y;
   }
+}
+
+template <int B>
+__device__ __forceinline__ float magic_of() {
+  return kMagic + (float)(1 << (B - 1));
+}
+
+// Head units of width B.
+template <int B, bool FULL>
+__device__ __forceinline__ void requant_head(const Ctx<FULL>& c, uint8_t* dst, const float4& icv) {
+  const float2 ic[4] = {dup(icv.x), dup(icv.y), dup(icv.z), dup(icv.w)};
+  const uint32_t rb = row_bytes_of<B>(c.dv());
+  uint8_t* row0 = dst + 2u * (c.dk() + c.dv()) + (uint32_t)c.row0() * rb;
+  const float2* ir2 = reinterpret_cast<const float2*>(sp<float>(S_IR) + c.row0());
+  const bool act = c.act();
+  const int lane = c.lane;
+  sweep(c.tm, c.nch(), [&](int ch, float2 (&v)[8]) {
+#pragma unroll
+    for (int pr = 0; pr < 2; ++pr) {
+      float ya[4], yb[4];
+      quant_pair(v + 4 * pr, ir2[2 * ch + pr], ic, magic_of<B>(), ya, yb);
+      uint8_t* ra = row0 + (uint32_t)(4 * ch + 2 * pr) * rb;
+      store4<B>(ra, lane, ya, act);
+      store4<B>(ra + rb, lane, yb, act);
+    }
+  });
+}
+
+// Key-row units: per-row width (chunk-level dispatch when the chunk has one width).
+__device__ __forceinline__ void store_row_rt(int b, uint8_t* row, int lane, const float2* g,
+                                             bool odd, float ir, const float (&ic)[4], bool act) {
+  float s[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) s[e] = odd ? g[e].y : g[e].x;
+  if (b == 16) {
+    store4_f16(row, lane, s, act);
+    return;
+  }
+  const float mg = kMagic + (float)(1 << (b - 1));
+  float y[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) y[e] = __fmaf_rn(__fmul_rn(s[e], ir), ic[e], mg);
+  switch (b) {
+    case 2: store4<2>(row, lane, y, act); break;
+    case 4: store4<4>(row, lane, y, act); break;
+    case 6: store4<6>(row, lane, y, act); break;
+    default: store4<8>(row, lane, y, act); break;
+  }
+}
+
+template <int B>
+__device__ __forceinline__ void requant_chunk_uniform(const float2 (&v)[8], const uint32_t (&ds)[4],
+                                                      uint8_t* dst, const float2* ir2, int ch,
+                                                      const float2 (&ic)[4], int lane, bool act) {
+#pragma unroll
+  for (int pr = 0; pr < 2; ++pr) {
+    float ya[4], yb[4];
+    quant_pair(v + 4 * pr, ir2[2 * ch + pr], ic, magic_of<B>(), ya, yb);
+    store4<B>(dst + rd_off(ds[2 * pr]), lane, ya, act);
+    store4<B>(dst + rd_off(ds[2 * pr + 1]), lane, yb, act);
+  }
+}
+
+template <bool FULL>
+__device__ __forceinline__ void requant_rows(const Ctx<FULL>& c, uint8_t* dst, const float4& icv) {
+  const float2 ic2[4] = {dup(icv.x), dup(icv.y), dup(icv.z), dup(icv.w)};
+  const float ic[4] = {icv.x, icv.y, icv.z, icv.w};
+  const float* irs = sp<float>(S_IR) + c.row0();
+  const float2* ir2 = reinterpret_cast<const float2*>(irs);
+  const uint4* rd4 = reinterpret_cast<const uint4*>(sp<uint32_t>(S_RD) + c.row0());
+  const bool act = c.act();
+  const int lane = c.lane;
+  sweep(c.tm, c.nch(), [&](int ch, float2 (&v)[8]) {
+    const uint4 d = rd4[ch];
+    const uint32_t ds[4] = {d.x, d.y, d.z, d.w};
+    const int b0 = rd_width(ds[0]);
+    const bool uni = b0 == rd_width(ds[1]) && b0 == rd_width(ds[2]) && b0 == rd_width(ds[3]);
+    if (uni && b0 == 2) {
+      requant_chunk_uniform<2>(v, ds, dst, ir2, ch, ic2, lane, act);
+    } else if (uni && b0 == 4) {
+      requant_chunk_uniform<4>(v, ds, dst, ir2, ch, ic2, lane, act);
+    } else if (uni && b0 == 6) {
+      requant_chunk_uniform<6>(v, ds, dst, ir2, ch, ic2, lane, act);
+    } else if (uni && b0 == 8) {
+      requant_chunk_uniform<8>(v, ds, dst, ir2, ch, ic2, lane, act);
+    } else {
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+        store_row_rt(rd_width(ds[r]), dst + rd_off(ds[r]), lane, v + 4 * (r >> 1), r & 1,
+                     irs[4 * ch + r], ic, act);
+    }
+  });
 }
 
 // fp16 head: round and store the updated tile.
 template <bool FULL>
 __device__ __forceinline__ void store_pivot(const Ctx<FULL>& c, uint8_t* dst) {
-  if (!c.wact()) return;
-  const Geo<MODE_PIVOT> geo(c);
-#pragma unroll 1
-  for (int ch = 0; ch < kChunks; ++ch) {
-    float2 v[8];
-    tmem_ld16x2(c.tm + 16 * ch, v);
+  const uint32_t rb = 2u * c.dv();
+  uint8_t* row0 = dst + (uint32_t)c.row0() * rb;
+  const bool act = c.act();
+  const int lane = c.lane;
+  sweep(c.tm, c.nch(), [&](int ch, float2 (&v)[8]) {
 #pragma unroll
-    for (int r = 0; r < 4; ++r)
-      store4_f16x2(dst + geo.off(c.row0() + 4 * ch + r), c.lane, v[2 * r], v[2 * r + 1], c.act());
-  }
+    for (int r = 0; r < 4; ++r) {
+      const float2* g = v + 4 * (r >> 1);
+      const float s[4] = {(r & 1) ? g[0].y : g[0].x, (r & 1) ? g[1].y : g[1].x,
+                          (r & 1) ? g[2].y : g[2].x, (r & 1) ? g[3].y : g[3].x};
+      store4_f16(row0 + (uint32_t)(4 * ch + r) * rb, lane, s, act);
+    }
+  });
 }
 
 __device__ __forceinline__ void nan_out(float* out, int dv, int tid) {
   if (tid < dv) out[tid] = __int_as_float(0x7fc00000);
 }
 
-template <int GATE, int IO, bool WANT_STATE, bool FULL>
-__global__ void __launch_bounds__(kThreads, 3) k_decode(const StepArgs a) {
-  const int nst = a.n_stages;
-  const DPlan P(a.dk, a.dv, IO, GATE, a.per_row, a.stage_bytes, a.H, nst);
-  uint64_t* bars = sp<uint64_t>(OFF_BAR);
+template <int GATE, int IO, bool WS, bool FULL>
+__global__ void __launch_bounds__(kT, kMaxCtasPerSm) k_decode(const StepArgs a) {
+  const DPlan P(a.dk, a.dv, IO, GATE, a.per_row, a.stage_bytes, a.H);
+  uint64_t* bar = sp<uint64_t>(S_BAR);
   Ctx<FULL> c;
   c.tid = threadIdx.x;
   c.warp = c.tid >> 5;
@@ -459,37 +696,40 @@ __global__ void __launch_bounds__(kThreads, 3) k_decode(const StepArgs a) {
   c.dk_ = a.dk;
   c.dv_ = a.dv;
   c.act_ = 4 * c.lane < a.dv;
-  c.wact_ = c.warp * kRows < a.dk;
+  {
+    const int rows = a.dk - c.warp * kRW;
+    c.nch_ = rows <= 0 ? 0 : (rows >= kRW ? kMaxCh : rows / 4);
+  }
   const int H = a.H, B = a.batch, dk = c.dk(), dv = c.dv(), tid = c.tid;
   const int n_items = B * H;
   const int stride = gridDim.x;
 
   if (c.warp == 0) {
-    tmem_alloc(sp<uint32_t>(OFF_TMEM), kTmemCols);
+    tmem_alloc(sp<uint32_t>(S_TMEM), kTmemCols);
     tmem_relinquish();
   }
   if (tid == 0) {
-    for (int s = 0; s < nst; ++s) mbar_init(&bars[s], 1);
+    mbar_init(bar, 1);
     fence_mbar_init();
   }
-  if (tid < 16) sp<int>(OFF_FLAGS)[tid] = 0;
+  if (tid < 16) sp<int>(S_FLAGS)[tid] = 0;
   HeadDesc* htab = reinterpret_cast<HeadDesc*>(smem + P.tab);
   int32_t* otab = reinterpret_cast<int32_t*>(smem + P.tab + 16u * H);
-  for (int h = tid; h < H; h += kThreads) {
+  for (int h = tid; h < H; h += kT) {
     htab[h] = a.heads[h];
     otab[h] = a.order[h];
   }
   tmem_fence_before_sync();
   __syncthreads();
   tmem_fence_after_sync();
-  const uint32_t tbase = *sp<uint32_t>(OFF_TMEM);
-  c.tm = tbase + ((uint32_t)(32 * (c.warp & 3)) << 16) + 64u * (uint32_t)(c.warp >> 2);
+  const uint32_t tbase = *sp<uint32_t>(S_TMEM);
+  c.tm = tbase + ((uint32_t)(32 * c.warp) << 16);
 
   // Items run head-major in the order of otab: item = hh * B + b. The last warp stages them;
   // its cursors advance by the grid stride without divisions.
-  Meta* meta = sp<Meta>(OFF_META);
-  int* flag_base = sp<int>(OFF_FLAGS);
-  const bool producer = c.warp == kWarps - 1;
+  Meta* meta = sp<Meta>(S_META);
+  int* flag_base = sp<int>(S_FLAGS);
+  const bool producer = c.warp == kW - 1;
   const int first = blockIdx.x;
   const int step_hh = stride / B, step_b = stride - step_hh * B;
   struct Cursor {
@@ -504,10 +744,9 @@ __global__ void __launch_bounds__(kThreads, 3) k_decode(const StepArgs a) {
       ++k.hh;
     }
   };
-  Cursor next_issue{first, first / B, first % B};  // the item to stage next
-  Cursor next_meta = next_issue;                    // the item whose words to fetch next
-  // Producer lanes 0..2: async copies of an item's slot index, beta and (scalar) alpha.
-  auto fetch_meta = [&](Cursor& k) {
+  Cursor next_issue{first, first / B, first % B};
+  Cursor next_meta = next_issue;
+  auto fetch_meta = [&](Cursor& k) {  // producer lanes 0..2: the item's slot, beta, alpha
     if (c.lane < 3) {
       const int io = k.b * H + otab[k.hh];
       if (c.lane == 0) cp_async4(&meta->slot, a.slot_idx + k.b);
@@ -517,14 +756,13 @@ __global__ void __launch_bounds__(kThreads, 3) k_decode(const StepArgs a) {
     }
     advance(k);
   };
-  // Producer warp: stage an item into stage s (its words are in *meta). Lane 0 clears the
-  // item's flag words, writes the header and arrives on the stage's mbarrier with the byte
-  // count (the arrive publishes both); lanes 1..6 issue one bulk copy each.
-  auto issue = [&](Cursor& k, int s, int* nflags) {
+  // Producer warp: stage an item (its words are in *meta). Lane 0 clears the item's flag words,
+  // writes the header and arrives on the mbarrier with the byte count; lanes 1..6 issue one
+  // bulk copy each.
+  auto issue = [&](Cursor& k, int* nflags) {
     if (c.lane < 3) cp_async_wait_all();
     __syncwarp();
-    uint8_t* st = smem + OFF_STAGE + s * P.stage;
-    uint64_t* bar = &bars[s];
+    uint8_t* st = smem + S_STAGE;
     const int h = otab[k.hh], io = k.b * H + h;
     const HeadDesc hd = htab[h];
     const Meta m = *meta;
@@ -537,7 +775,7 @@ __global__ void __launch_bounds__(kThreads, 3) k_decode(const StepArgs a) {
       *reinterpret_cast<int4*>(shdr) = make_int4(valid, m.slot, k.b, h);
       *(reinterpret_cast<int4*>(shdr) + 1) =
           make_int4(__float_as_int(m.beta), __float_as_int(GATE == 0 ? m.alpha : 0.f),
-                    hd.pivot_head ? (int)MODE_PIVOT : (int)hd.width, (int)hd.off);
+                    hd.pivot_head ? MODE_PIVOT : (int)hd.width, (int)hd.off);
       mbar_arrive_expect_tx(bar, valid ? 2 * kb + vb + ab + rb + hd.bytes : 0u);
     }
     if (valid && c.lane >= 1 && c.lane <= 6) {
@@ -549,7 +787,7 @@ __global__ void __launch_bounds__(kThreads, 3) k_decode(const StepArgs a) {
         case 2: dst += P.q_off, src = static_cast<const uint8_t*>(a.q) + (size_t)io * kb, n = kb; break;
         case 3: dst += P.v_off, src = static_cast<const uint8_t*>(a.v) + (size_t)io * vb, n = vb; break;
         case 4: dst += P.al_off, src = reinterpret_cast<const uint8_t*>(a.alpha + (size_t)io * dk), n = ab; break;
-        case 5: dst += P.rt_off, src = reinterpret_cast<const uint8_t*>(a.rows + (size_t)h * dk), n = rb; break;
+        case 5: dst += P.rt_off, src = reinterpret_cast<const uint8_t*>(a.srows + (size_t)h * dk), n = rb; break;
         default: dst += P.blk_off, src = a.pool + (size_t)m.slot * a.slot_bytes + hd.off, n = hd.bytes; break;
       }
       if (n) bulk_load(dst, src, n, bar);
@@ -558,93 +796,93 @@ __global__ void __launch_bounds__(kThreads, 3) k_decode(const StepArgs a) {
     advance(k);
   };
 
-  if (producer) {  // the first n_stages items in flight, the next one's words on their way
-    for (int s = 0; s < nst && next_issue.item < n_items; ++s) {
-      fetch_meta(next_meta);
-      issue(next_issue, s, flag_base + 4 * s);
-    }
+  if (producer && next_issue.item < n_items) {
+    fetch_meta(next_meta);
+    issue(next_issue, flag_base);
     if (next_meta.item < n_items) fetch_meta(next_meta);
   }
 
   int it = 0;
   bool timed_out = false;
+  const uint8_t* st = smem + S_STAGE;
+  const uint8_t* blk = st + P.blk_off;
   for (int item = first; item < n_items; item += stride, ++it) {
-    // warp-uniform, so the warp-collective tensor-memory instructions below never diverge
-    const int s = nst == 1 ? 0 : (it & 1);
-    const uint32_t phase = (uint32_t)(nst == 1 ? it : it >> 1) & 1u;
-    const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars[s], phase));
+    const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar, (uint32_t)it & 1u));
     c.flags = flag_base + 4 * (it & 3);
-    const uint8_t* st = smem + OFF_STAGE + s * P.stage;
-    c.blk = st + P.blk_off;
     StageHdr hdr = *reinterpret_cast<const StageHdr*>(st);
     if (!ok) hdr.valid = 0;
     const int io = hdr.b * H + hdr.h;
-    const bool pivot_head = hdr.mode == MODE_PIVOT;
+    const int mode = hdr.mode;
+    const bool pivot_head = mode == MODE_PIVOT;
 
-    // ---- setup (each warp its own rows' factors and k.q partial; warps 0 and 1 the column
-    // data) and pass A ----
+    // ---- setup: thread t takes processing row t (its factors) and every lane its four
+    // columns' old scale and v, before the stage is handed back ----
+    float4 cv = make_float4(1.f, 1.f, 1.f, 1.f), vv = make_float4(0.f, 0.f, 0.f, 0.f);
+    float4 icv = make_float4(1.f, 1.f, 1.f, 1.f);
     if (hdr.valid) {
-      const uint8_t* kq = st + P.k_off;
-      const uint8_t* qq = st + P.q_off;
       bool bad_in = false;
       float kqp = 0.f;
-      if (c.wact() && c.lane < kRows) {
-        const int i = c.row0() + c.lane;
-        uint32_t desc = 0;
+      const int p = tid;
+      if (p < dk) {
+        uint32_t d;
         if (a.per_row) {
-          desc = reinterpret_cast<const uint32_t*>(st + P.rt_off)[i];
-          c.rowtab()[i] = desc;
+          d = reinterpret_cast<const uint32_t*>(st + P.rt_off)[p];
+        } else {
+          const uint32_t off = pivot_head ? (uint32_t)p * 2u * dv
+                                          : 2u * (dk + dv) + (uint32_t)p * dv * mode / 8u;
+          d = (uint32_t)p << 24 | off << 8 | (uint32_t)mode;
         }
-        const float ki = ld_io(kq, IO, i), qi = ld_io(qq, IO, i);
+        sp<uint32_t>(S_RD)[p] = d;
+        const int i = rd_row(d);
+        const float ki = ld_io(st + P.k_off, IO, i), qi = ld_io(st + P.q_off, IO, i);
         const float ai = GATE == 0 ? hdr.alpha : reinterpret_cast<const float*>(st + P.al_off)[i];
         bad_in |= !isfinite(ki) || !isfinite(qi) || !isfinite(ai);
-        const bool qrow = !pivot_head && (!a.per_row || row_width(desc) != 16);
-        const float A = qrow ? ai * __half2float(reinterpret_cast<const __half*>(c.blk)[i]) : ai;
-        c.rowG()[i] = make_float4(A * ki, A * ki, A * qi, A * qi);
-        c.rowU()[i] = make_float4(A, A, ki, ki);
+        const float A = rd_width(d) != 16 ? ai * __half2float(reinterpret_cast<const __half*>(blk)[i]) : ai;
+        float* gkq = sp<float>(S_GKQ) + 4 * (p >> 1) + (p & 1);
+        gkq[0] = A * ki;
+        gkq[2] = A * qi;
+        float* akp = sp<float>(S_AK) + 4 * (p >> 1) + (p & 1);
+        akp[0] = A;
+        akp[2] = ki;
         kqp = ki * qi;
       }
       kqp = warp_sum(kqp);
-      if (c.lane == 0) sp<float>(OFF_KQP)[c.warp] = kqp;
-      if (c.warp == 0) {
-        float4 cv = make_float4(1.f, 1.f, 1.f, 1.f);
-        if (c.act() && !pivot_head) {
-          const uint2 ch = reinterpret_cast<const uint2*>(c.blk + 2 * dk)[c.lane];
+      if (c.lane == 0) sp<float>(S_KQ)[c.warp] = kqp;
+      if (c.act()) {
+        if (!pivot_head) {
+          const uint2 ch = reinterpret_cast<const uint2*>(blk + 2 * dk)[c.lane];
           const float2 a01 = __half22float2(*reinterpret_cast<const __half2*>(&ch.x));
           const float2 a23 = __half22float2(*reinterpret_cast<const __half2*>(&ch.y));
           cv = make_float4(a01.x, a01.y, a23.x, a23.y);
+          if (mode == MODE_ROWS)
+            icv = make_float4(rcp_f16val(cv.x), rcp_f16val(cv.y), rcp_f16val(cv.z), rcp_f16val(cv.w));
         }
-        sp<float4>(OFF_COLC)[c.lane] = cv;
-        bad_in |= !isfinite(hdr.beta) || (GATE == 0 && !isfinite(hdr.alpha));
-      } else if (c.warp == 1) {
-        float4 vv = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (c.act()) {
-          const uint8_t* vq = st + P.v_off;
-          vv = make_float4(ld_io(vq, IO, 4 * c.lane), ld_io(vq, IO, 4 * c.lane + 1),
-                           ld_io(vq, IO, 4 * c.lane + 2), ld_io(vq, IO, 4 * c.lane + 3));
+        const uint8_t* vq = st + P.v_off;
+        vv = make_float4(ld_io(vq, IO, 4 * c.lane), ld_io(vq, IO, 4 * c.lane + 1),
+                         ld_io(vq, IO, 4 * c.lane + 2), ld_io(vq, IO, 4 * c.lane + 3));
+        if (c.warp == 0)
           bad_in |= !(isfinite(vv.x) && isfinite(vv.y) && isfinite(vv.z) && isfinite(vv.w));
-        }
-        sp<float4>(OFF_COLV)[c.lane] = vv;
       }
+      if (tid == 0) bad_in |= !isfinite(hdr.beta) || (GATE == 0 && !isfinite(hdr.alpha));
       if (bad_in) atomicOr(&c.flags[F_INPUT], 1);
       __syncwarp();
-      switch (hdr.mode) {
-        case MODE_W2: pass_a<MODE_W2>(c); break;
-        case MODE_W4: pass_a<MODE_W4>(c); break;
-        case MODE_W6: pass_a<MODE_W6>(c); break;
-        case MODE_W8: pass_a<MODE_W8>(c); break;
-        case MODE_PIVOT: pass_a<MODE_PIVOT>(c); break;
-        default: pass_a<MODE_ROWS>(c); break;
+      switch (mode) {
+        case 2: pass_a_head<2>(c, blk); break;
+        case 4: pass_a_head<4>(c, blk); break;
+        case 6: pass_a_head<6>(c, blk); break;
+        case 8: pass_a_head<8>(c, blk); break;
+        case MODE_PIVOT: pass_a_head<16>(c, blk); break;
+        default: pass_a_rows(c, blk, icv); break;
       }
       tmem_wait_st();
     }
-    // barrier 1: partial dot products, input flags; the stage is free afterwards
+    // barrier 1: partial dot products and flags; the stage is free afterwards
     if (__syncthreads_or(!ok)) {
       timed_out = true;
       break;
     }
-    if (producer && next_issue.item < n_items) {  // refill this stage (item + nst strides)
-      issue(next_issue, s, flag_base + 4 * ((it + nst) & 3));
+    if (producer && next_issue.item < n_items) {  // stage the next item
+      issue(next_issue, flag_base + 4 * ((it + 1) & 3));
       if (next_meta.item < n_items) fetch_meta(next_meta);
     }
     float* out = a.out + (size_t)io * dv;
@@ -660,28 +898,26 @@ __global__ void __launch_bounds__(kThreads, 3) k_decode(const StepArgs a) {
     }
 
     // ---- b, o ----
-    const float4 cv = sp<float4>(OFF_COLC)[c.lane];
     float4 bv;
     {
-      const float4 kq0 = sp<float4>(OFF_KQP)[0], kq1 = sp<float4>(OFF_KQP)[1];
-      const float kqv = ((kq0.x + kq0.y) + (kq0.z + kq0.w)) + ((kq1.x + kq1.y) + (kq1.z + kq1.w));
-      const float4 vv = sp<float4>(OFF_COLV)[c.lane];
-      const float4 U = sum8(sp<float>(OFF_REDA), 2 * kMaxD, c.lane);
+      const float4 kq4 = *sp<float4>(S_KQ);
+      const float kqv = (kq4.x + kq4.y) + (kq4.z + kq4.w);
+      const float4 U = sum4(sp<float>(S_REDU), c.lane);
       const float beta = hdr.beta;
       bv = make_float4(beta * (vv.x - cv.x * U.x), beta * (vv.y - cv.y * U.y),
                        beta * (vv.z - cv.z * U.z), beta * (vv.w - cv.w * U.w));
       if (c.warp == 0 && c.act()) {
-        const float4 Pp = sum8(sp<float>(OFF_REDA) + kMaxD, 2 * kMaxD, c.lane);
+        const float4 Pp = sum4(sp<float>(S_REDP), c.lane);
         *reinterpret_cast<float4*>(out + 4 * c.lane) =
             make_float4(__fmaf_rn(bv.x, kqv, cv.x * Pp.x), __fmaf_rn(bv.y, kqv, cv.y * Pp.y),
                         __fmaf_rn(bv.z, kqv, cv.z * Pp.z), __fmaf_rn(bv.w, kqv, cv.w * Pp.w));
       }
     }
-    float* s_new = WANT_STATE ? a.s_new + (size_t)io * dk * dv : nullptr;
+    float* s_new = WS ? a.s_new + (size_t)io * dk * dv : nullptr;
     uint8_t* dst = a.pool + (size_t)hdr.slot * a.slot_bytes + hdr.off;
 
     if (pivot_head) {
-      pass_b(c, cv, bv, s_new, 1, false);
+      pass_b<1, WS>(c, cv, bv, s_new);
       __syncthreads();
       if (c.flags[F_RANGE]) {
         if (tid == 0) atomicOr(a.flag, SQ_FLAG_RANGE_BIT);
@@ -692,40 +928,40 @@ __global__ void __launch_bounds__(kThreads, 3) k_decode(const StepArgs a) {
     }
 
     // ---- refit: alternating row / column max-abs passes ----
-    pass_b(c, cv, bv, s_new, a.per_row ? 2 : 0, true);
-    float r = row_scales(c, hdr.mode, true);
-    col_pass(c, sp<float>(OFF_REDC));
+    if (mode == MODE_ROWS)
+      pass_b<2, WS>(c, cv, bv, s_new);
+    else
+      pass_b<0, WS>(c, cv, bv, s_new);
+    float r = row_scales(c, true);
+    col_pass(c, sp<float>(S_REDC));
     __syncthreads();  // barrier 2
-    float4 cm = max8(sp<float>(OFF_REDC), c.lane);
+    float4 cm = max4(sp<float>(S_REDC), c.lane);
     for (int f = 1; f < a.fit_iters; ++f) {
-      const float4 icv = make_float4(rcp_approx(cm.x), rcp_approx(cm.y), rcp_approx(cm.z), rcp_approx(cm.w));
-      row_pass(c, icv);
-      r = row_scales(c, hdr.mode, false);
-      float* red = sp<float>(OFF_REDC) + (f & 1) * kWarps * kMaxD;
+      row_pass(c, make_float4(rcp_approx(cm.x), rcp_approx(cm.y), rcp_approx(cm.z), rcp_approx(cm.w)));
+      r = row_scales(c, false);
+      float* red = sp<float>(S_REDC) + (f & 1) * kW * kMaxD;
       col_pass(c, red);
       __syncthreads();  // barrier 3 (fit_iters = 2)
-      cm = max8(red, c.lane);
+      cm = max4(red, c.lane);
     }
     if (c.flags[F_RANGE]) {
       if (tid == 0) atomicOr(a.flag, SQ_FLAG_RANGE_BIT);
       continue;
     }
-    switch (hdr.mode) {
-      case MODE_W2: requant<MODE_W2>(c, dst, cm, r); break;
-      case MODE_W4: requant<MODE_W4>(c, dst, cm, r); break;
-      case MODE_W6: requant<MODE_W6>(c, dst, cm, r); break;
-      case MODE_W8: requant<MODE_W8>(c, dst, cm, r); break;
-      default: requant<MODE_ROWS>(c, dst, cm, r); break;
+    const float4 icn = store_scales(c, dst, cm, r);
+    switch (mode) {
+      case 2: requant_head<2>(c, dst, icn); break;
+      case 4: requant_head<4>(c, dst, icn); break;
+      case 6: requant_head<6>(c, dst, icn); break;
+      case 8: requant_head<8>(c, dst, icn); break;
+      default: requant_rows(c, dst, icn); break;
     }
   }
 
   if (timed_out) {
     if (tid == 0) atomicOr(a.flag, SQ_FLAG_TIMEOUT_BIT);
     // let copies still in flight land before the CTA exits
-    const int s = nst == 1 ? 0 : (it & 1);
-    mbar_wait_bounded(&bars[s], (uint32_t)(nst == 1 ? it : it >> 1) & 1u);
-    const int item = first + it * stride;
-    if (nst == 2 && item + stride < n_items) mbar_wait_bounded(&bars[s ^ 1], (uint32_t)((it + 1) >> 1) & 1u);
+    mbar_wait_bounded(bar, (uint32_t)it & 1u);
     if (producer && c.lane < 3) cp_async_wait_all();
   }
   tmem_fence_before_sync();
@@ -736,7 +972,7 @@ __global__ void __launch_bounds__(kThreads, 3) k_decode(const StepArgs a) {
   }
 }
 
-// Resident CTAs of kThreads threads per SM, from the registers and shared memory a CTA holds.
+// Resident CTAs of kT threads per SM, from the registers and shared memory a CTA holds.
 cudaError_t resident_ctas(const void* fn, uint32_t smem_bytes, int* per_sm) {
   cudaFuncAttributes fa;
   cudaError_t e = cudaFuncGetAttributes(&fa, fn);
@@ -747,8 +983,8 @@ cudaError_t resident_ctas(const void* fn, uint32_t smem_bytes, int* per_sm) {
   if ((e = cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&thr_sm, cudaDevAttrMaxThreadsPerMultiProcessor, dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev)) != cudaSuccess) return e;
-  const int regs_cta = ((fa.numRegs + 7) / 8 * 8) * kThreads;  // allocated per warp in units of 8 per thread
-  int n = thr_sm / kThreads;
+  const int regs_cta = ((fa.numRegs + 7) / 8 * 8) * kT;  // allocated per warp in units of 8 per thread
+  int n = thr_sm / kT;
   if (regs_cta > 0 && regs_sm / regs_cta < n) n = regs_sm / regs_cta;
   const int smem_cta = (int)smem_bytes + (int)fa.sharedSizeBytes + reserved;
   if (smem_sm / smem_cta < n) n = smem_sm / smem_cta;
@@ -759,33 +995,23 @@ cudaError_t resident_ctas(const void* fn, uint32_t smem_bytes, int* per_sm) {
 template <int GATE, int IO, bool WS, bool FULL>
 cudaError_t launch_t(const StepArgs& a, int num_sms, cudaStream_t st) {
   auto fn = k_decode<GATE, IO, WS, FULL>;
-  // Two stages where they still leave three CTAs on an SM, else one. Shared memory of at least
-  // a fifth of the SM's keeps at most four CTAs on an SM, so the tensor-memory allocations
-  // (128 columns each) always fit. CTAs per SM come from the kernel's registers and shared
-  // memory: the runtime's occupancy query answers 1 for kernels that allocate tensor memory.
-  StepArgs b = a;
-  uint32_t smem_bytes = 0;
+  // Shared memory of at least a fifth of the SM's keeps at most four CTAs on an SM, so the
+  // tensor-memory allocations (128 columns each) always fit. CTAs per SM come from the
+  // kernel's registers and shared memory: the runtime's occupancy query answers 1 for kernels
+  // that allocate tensor memory.
+  const DPlan P(a.dk, a.dv, IO, GATE, a.per_row, a.stage_bytes, a.H);
+  const uint32_t smem_bytes = P.total > 47u * 1024u ? P.total : 47u * 1024u;
   int per_sm = 0;
-  for (int nst = 2; nst >= 1; --nst) {  // the most CTAs per SM, then the most stages
-    const DPlan P(a.dk, a.dv, IO, GATE, a.per_row, a.stage_bytes, a.H, nst);
-    const uint32_t sb = P.total > 47u * 1024u ? P.total : 47u * 1024u;
-    int n = 0;
-    const cudaError_t e = resident_ctas(reinterpret_cast<const void*>(fn), sb, &n);
-    if (e != cudaSuccess) return e;
-    if (n > kMaxCtasPerSm) n = kMaxCtasPerSm;
-    if (n > per_sm) {
-      per_sm = n;
-      smem_bytes = sb;
-      b.n_stages = nst;
-    }
-  }
-  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
+  cudaError_t e = resident_ctas(reinterpret_cast<const void*>(fn), smem_bytes, &per_sm);
+  if (e != cudaSuccess) return e;
+  if (per_sm > kMaxCtasPerSm) per_sm = kMaxCtasPerSm;
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
   if (e != cudaSuccess) return e;
   const int items = a.batch * a.H;
   int grid = num_sms * per_sm;
   if (grid > items) grid = items;
   if (grid < 1) return cudaSuccess;
-  fn<<<grid, kThreads, smem_bytes, st>>>(b);
+  fn<<<grid, kT, smem_bytes, st>>>(a);
   return cudaGetLastError();
 }
 

@@ -41,6 +41,8 @@ struct StepArgs {
   float* s_new;  // optional fp32 state after the update (tests)
   const HeadDesc* heads;
   const uint32_t* rows;
+  const uint32_t* srows;  // key-row units: [H][d_k] row descriptors in processing order
+                          // (original row << 24 | byte offset << 8 | width), rows grouped by width
   const int32_t* order;  // heads sorted by width: items run head-major in this order
   int32_t H, dk, dv, fit_iters;
   int32_t per_row;       // 1: key-row units (the row table is staged with each head block)
