@@ -685,9 +685,11 @@ __device__ __forceinline__ void nan_out(float* out, int dv, int tid) {
   if (tid < dv) out[tid] = __int_as_float(0x7fc00000);
 }
 
-template <int GATE, int IO, bool WS, bool FULL>
+// ROWS: key-row units (per-row widths; every head block has row and column scales); else head
+// units (one width per head, fp16 pivot heads).
+template <int GATE, int IO, bool WS, bool FULL, bool ROWS>
 __global__ void __launch_bounds__(kT, kMaxCtasPerSm) k_decode(const StepArgs a) {
-  const DPlan P(a.dk, a.dv, IO, GATE, a.per_row, a.stage_bytes, a.H);
+  const DPlan P(a.dk, a.dv, IO, GATE, ROWS, a.stage_bytes, a.H);
   uint64_t* bar = sp<uint64_t>(S_BAR);
   Ctx<FULL> c;
   c.tid = threadIdx.x;
@@ -768,7 +770,7 @@ __global__ void __launch_bounds__(kT, kMaxCtasPerSm) k_decode(const StepArgs a) 
     const Meta m = *meta;
     const bool valid = m.slot >= 0 && m.slot < a.n_slots;
     const uint32_t kb = (uint32_t)dk * P.esz, vb = (uint32_t)dv * P.esz;
-    const uint32_t ab = GATE == 1 ? 4u * dk : 0u, rb = a.per_row ? 4u * dk : 0u;
+    const uint32_t ab = GATE == 1 ? 4u * dk : 0u, rb = ROWS ? 4u * dk : 0u;
     if (c.lane == 0) {
       nflags[F_INPUT] = nflags[F_RANGE] = 0;
       StageHdr* shdr = reinterpret_cast<StageHdr*>(st);
@@ -812,8 +814,8 @@ __global__ void __launch_bounds__(kT, kMaxCtasPerSm) k_decode(const StepArgs a) 
     StageHdr hdr = *reinterpret_cast<const StageHdr*>(st);
     if (!ok) hdr.valid = 0;
     const int io = hdr.b * H + hdr.h;
-    const int mode = hdr.mode;
-    const bool pivot_head = mode == MODE_PIVOT;
+    const int mode = ROWS ? MODE_ROWS : hdr.mode;
+    const bool pivot_head = !ROWS && mode == MODE_PIVOT;
 
     // ---- setup: thread t takes processing row t (its factors) and every lane its four
     // columns' old scale and v, before the stage is handed back ----
@@ -825,7 +827,7 @@ __global__ void __launch_bounds__(kT, kMaxCtasPerSm) k_decode(const StepArgs a) 
       const int p = tid;
       if (p < dk) {
         uint32_t d;
-        if (a.per_row) {
+        if (ROWS) {
           d = reinterpret_cast<const uint32_t*>(st + P.rt_off)[p];
         } else {
           const uint32_t off = pivot_head ? (uint32_t)p * 2u * dv
@@ -854,7 +856,7 @@ __global__ void __launch_bounds__(kT, kMaxCtasPerSm) k_decode(const StepArgs a) 
           const float2 a01 = __half22float2(*reinterpret_cast<const __half2*>(&ch.x));
           const float2 a23 = __half22float2(*reinterpret_cast<const __half2*>(&ch.y));
           cv = make_float4(a01.x, a01.y, a23.x, a23.y);
-          if (mode == MODE_ROWS)
+          if (ROWS)
             icv = make_float4(rcp_f16val(cv.x), rcp_f16val(cv.y), rcp_f16val(cv.z), rcp_f16val(cv.w));
         }
         const uint8_t* vq = st + P.v_off;
@@ -866,13 +868,16 @@ __global__ void __launch_bounds__(kT, kMaxCtasPerSm) k_decode(const StepArgs a) 
       if (tid == 0) bad_in |= !isfinite(hdr.beta) || (GATE == 0 && !isfinite(hdr.alpha));
       if (bad_in) atomicOr(&c.flags[F_INPUT], 1);
       __syncwarp();
-      switch (mode) {
-        case 2: pass_a_head<2>(c, blk); break;
-        case 4: pass_a_head<4>(c, blk); break;
-        case 6: pass_a_head<6>(c, blk); break;
-        case 8: pass_a_head<8>(c, blk); break;
-        case MODE_PIVOT: pass_a_head<16>(c, blk); break;
-        default: pass_a_rows(c, blk, icv); break;
+      if (ROWS) {
+        pass_a_rows(c, blk, icv);
+      } else {
+        switch (mode) {
+          case 2: pass_a_head<2>(c, blk); break;
+          case 4: pass_a_head<4>(c, blk); break;
+          case 6: pass_a_head<6>(c, blk); break;
+          case 8: pass_a_head<8>(c, blk); break;
+          default: pass_a_head<16>(c, blk); break;
+        }
       }
       tmem_wait_st();
     }
@@ -916,7 +921,7 @@ __global__ void __launch_bounds__(kT, kMaxCtasPerSm) k_decode(const StepArgs a) 
     float* s_new = WS ? a.s_new + (size_t)io * dk * dv : nullptr;
     uint8_t* dst = a.pool + (size_t)hdr.slot * a.slot_bytes + hdr.off;
 
-    if (pivot_head) {
+    if (!ROWS && pivot_head) {
       pass_b<1, WS>(c, cv, bv, s_new);
       __syncthreads();
       if (c.flags[F_RANGE]) {
@@ -928,10 +933,7 @@ __global__ void __launch_bounds__(kT, kMaxCtasPerSm) k_decode(const StepArgs a) 
     }
 
     // ---- refit: alternating row / column max-abs passes ----
-    if (mode == MODE_ROWS)
-      pass_b<2, WS>(c, cv, bv, s_new);
-    else
-      pass_b<0, WS>(c, cv, bv, s_new);
+    pass_b<ROWS ? 2 : 0, WS>(c, cv, bv, s_new);
     float r = row_scales(c, true);
     col_pass(c, sp<float>(S_REDC));
     __syncthreads();  // barrier 2
@@ -949,12 +951,15 @@ __global__ void __launch_bounds__(kT, kMaxCtasPerSm) k_decode(const StepArgs a) 
       continue;
     }
     const float4 icn = store_scales(c, dst, cm, r);
-    switch (mode) {
-      case 2: requant_head<2>(c, dst, icn); break;
-      case 4: requant_head<4>(c, dst, icn); break;
-      case 6: requant_head<6>(c, dst, icn); break;
-      case 8: requant_head<8>(c, dst, icn); break;
-      default: requant_rows(c, dst, icn); break;
+    if (ROWS) {
+      requant_rows(c, dst, icn);
+    } else {
+      switch (mode) {
+        case 2: requant_head<2>(c, dst, icn); break;
+        case 4: requant_head<4>(c, dst, icn); break;
+        case 6: requant_head<6>(c, dst, icn); break;
+        default: requant_head<8>(c, dst, icn); break;
+      }
     }
   }
 
@@ -992,9 +997,9 @@ cudaError_t resident_ctas(const void* fn, uint32_t smem_bytes, int* per_sm) {
   return cudaSuccess;
 }
 
-template <int GATE, int IO, bool WS, bool FULL>
+template <int GATE, int IO, bool WS, bool FULL, bool ROWS>
 cudaError_t launch_t(const StepArgs& a, int num_sms, cudaStream_t st) {
-  auto fn = k_decode<GATE, IO, WS, FULL>;
+  auto fn = k_decode<GATE, IO, WS, FULL, ROWS>;
   // Shared memory of at least a fifth of the SM's keeps at most four CTAs on an SM, so the
   // tensor-memory allocations (128 columns each) always fit. CTAs per SM come from the
   // kernel's registers and shared memory: the runtime's occupancy query answers 1 for kernels
@@ -1015,10 +1020,16 @@ cudaError_t launch_t(const StepArgs& a, int num_sms, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+// The 128 x 128 tile has its own compile-time-shaped kernels, except for the debug variant
+// that also writes the fp32 state.
 template <int GATE, int IO, bool WS>
 cudaError_t launch_shape(const StepArgs& a, int num_sms, cudaStream_t st) {
-  if (a.dk == kMaxD && a.dv == kMaxD) return launch_t<GATE, IO, WS, true>(a, num_sms, st);
-  return launch_t<GATE, IO, WS, false>(a, num_sms, st);
+  const bool full = !WS && a.dk == kMaxD && a.dv == kMaxD;
+  if (a.per_row)
+    return full ? launch_t<GATE, IO, false, true, true>(a, num_sms, st)
+                : launch_t<GATE, IO, WS, false, true>(a, num_sms, st);
+  return full ? launch_t<GATE, IO, false, true, false>(a, num_sms, st)
+              : launch_t<GATE, IO, WS, false, false>(a, num_sms, st);
 }
 
 }  // namespace
