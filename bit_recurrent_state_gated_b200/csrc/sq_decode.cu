@@ -35,6 +35,7 @@
 // S_ij / (r16_i c16_j) is at most Q (1 + 2^-10) in magnitude, less than Q + 1/2 for Q <= 127.
 // The state is the GPU's own fp32 update (fused multiply-adds), so its scales and codes are
 // compared with the oracle's within the stated agreement.
+#include "sq_pair.cuh"
 #include "sq_tile.cuh"
 
 namespace sq {
@@ -114,11 +115,6 @@ __device__ __forceinline__ T* sp(uint32_t off) {
   return reinterpret_cast<T*>(smem + off);
 }
 
-__device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
-__device__ __forceinline__ float2 lo(const float4& v) { return make_float2(v.x, v.y); }
-__device__ __forceinline__ float2 hi(const float4& v) { return make_float2(v.z, v.w); }
-__device__ __forceinline__ float2 dup(float a) { return make_float2(a, a); }
-
 __device__ __forceinline__ float max3abs(float a, float b, float c) {  // max(|a|, |b|, |c|)
   float d;
   asm("max.abs.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
@@ -136,13 +132,6 @@ __device__ __forceinline__ float rowmax_x(const float2* v) {
 __device__ __forceinline__ float rowmax_y(const float2* v) {
   return fmaxf(max3abs(v[0].y, v[1].y, v[2].y), fabsf(v[3].y));
 }
-
-__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(dst)), "l"(src)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 // ---- tensor memory, one chunk (16 columns) at a time, loads issued ahead of their use -------
 __device__ __forceinline__ void tm_issue(uint32_t taddr, uint32_t (&r)[16]) {
@@ -191,86 +180,6 @@ __device__ __forceinline__ void sweep(uint32_t tm, int nch, F&& body) {
     if (ch + 2 < nch) tm_issue(tm + 16u * (ch + 2), ra);
     body(ch + 1, w);
   }
-}
-
-// ---- unpack: the lane's four columns of two rows (a, b) as pairs (a_e, b_e) of exact codes --
-__device__ __forceinline__ float2 f2u(uint32_t x, uint32_t y) {
-  return make_float2(__uint_as_float(x), __uint_as_float(y));
-}
-
-template <int B>
-__device__ __forceinline__ void unpack_pair(const uint8_t* ra, const uint8_t* rb, int lane,
-                                            float2 (&x)[4]);
-
-template <>
-__device__ __forceinline__ void unpack_pair<2>(const uint8_t* ra, const uint8_t* rb, int lane,
-                                               float2 (&x)[4]) {
-  const uint32_t va = ra[lane], vb = rb[lane];  // f = 2^23 + u 4^e ; code = f 4^-e - (2^(23-2e) + 2)
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    const uint32_t m = 3u << (2 * e);
-    x[e] = __ffma2_rn(f2u(kMagicBits | (va & m), kMagicBits | (vb & m)),
-                      dup(1.0f / float(1u << (2 * e))), dup(-(float(1u << (23 - 2 * e)) + 2.0f)));
-  }
-}
-
-template <>
-__device__ __forceinline__ void unpack_pair<4>(const uint8_t* ra, const uint8_t* rb, int lane,
-                                               float2 (&x)[4]) {
-  const uint32_t va = reinterpret_cast<const uint16_t*>(ra)[lane];
-  const uint32_t vb = reinterpret_cast<const uint16_t*>(rb)[lane];
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    const uint32_t m = 15u << (4 * e);
-    x[e] = __ffma2_rn(f2u(kMagicBits | (va & m), kMagicBits | (vb & m)),
-                      dup(1.0f / float(1u << (4 * e))), dup(-(float(1u << (23 - 4 * e)) + 8.0f)));
-  }
-}
-
-__device__ __forceinline__ uint32_t bits24(const uint8_t* row, int lane) {  // 6-bit: lane's 24 bits
-  const int byte = 3 * lane;
-  const uint32_t* w = reinterpret_cast<const uint32_t*>(row + (byte & ~3));
-  return __funnelshift_r(w[0], w[1], (byte & 3) * 8);
-}
-
-template <>
-__device__ __forceinline__ void unpack_pair<6>(const uint8_t* ra, const uint8_t* rb, int lane,
-                                               float2 (&x)[4]) {
-  const uint32_t va = bits24(ra, lane), vb = bits24(rb, lane);
-  const uint32_t ha = va >> 12, hb = vb >> 12;
-  const float2 s1 = dup(1.0f / 64.0f);
-  const float2 o0 = dup(-(8388608.f + 32.f)), o1 = dup(-(131072.f + 32.f));
-  x[0] = __fadd2_rn(f2u(kMagicBits | (va & 63u), kMagicBits | (vb & 63u)), o0);
-  x[1] = __ffma2_rn(f2u(kMagicBits | (va & (63u << 6)), kMagicBits | (vb & (63u << 6))), s1, o1);
-  x[2] = __fadd2_rn(f2u(kMagicBits | (ha & 63u), kMagicBits | (hb & 63u)), o0);
-  x[3] = __ffma2_rn(f2u(kMagicBits | (ha & (63u << 6)), kMagicBits | (hb & (63u << 6))), s1, o1);
-}
-
-template <>
-__device__ __forceinline__ void unpack_pair<8>(const uint8_t* ra, const uint8_t* rb, int lane,
-                                               float2 (&x)[4]) {
-  const uint32_t va = reinterpret_cast<const uint32_t*>(ra)[lane];
-  const uint32_t vb = reinterpret_cast<const uint32_t*>(rb)[lane];
-  const float2 m = dup(-(kMagic + 128.f));
-#pragma unroll
-  for (int e = 0; e < 4; ++e)
-    x[e] = __fadd2_rn(f2u(__byte_perm(va, kMagicBits, 0x7540u + e),
-                          __byte_perm(vb, kMagicBits, 0x7540u + e)), m);
-}
-
-template <>
-__device__ __forceinline__ void unpack_pair<16>(const uint8_t* ra, const uint8_t* rb, int lane,
-                                                float2 (&x)[4]) {
-  // fp16 rows start on 4-byte boundaries: two 32-bit loads per row
-  const uint32_t* wa = reinterpret_cast<const uint32_t*>(ra) + 2 * lane;
-  const uint32_t* wb = reinterpret_cast<const uint32_t*>(rb) + 2 * lane;
-  const uint32_t a0 = wa[0], a1 = wa[1], b0 = wb[0], b1 = wb[1];
-  const __half2 ha0 = *reinterpret_cast<const __half2*>(&a0), ha1 = *reinterpret_cast<const __half2*>(&a1);
-  const __half2 hb0 = *reinterpret_cast<const __half2*>(&b0), hb1 = *reinterpret_cast<const __half2*>(&b1);
-  x[0] = f2(__low2float(ha0), __low2float(hb0));
-  x[1] = f2(__high2float(ha0), __high2float(hb0));
-  x[2] = f2(__low2float(ha1), __low2float(hb1));
-  x[3] = f2(__high2float(ha1), __high2float(hb1));
 }
 
 // Either row of a pair with its own width (key-row units, rows of two widths).
@@ -1032,6 +941,807 @@ cudaError_t launch_shape(const StepArgs& a, int num_sms, cudaStream_t st) {
               : launch_t<GATE, IO, WS, false, false>(a, num_sms, st);
 }
 
+
+// =============================================================================================
+// Windowed variant (LeapQuant news, 研究の概要: quantize only at the end of a window of tokens;
+// inside it the output comes from the frozen low-bit state plus the update held at high
+// precision; a few large entries are kept as high-precision "compensation" elements).
+//
+// The exact state inside a window is S_t = diag(g_t) (Sbar + sum_{s<t} k_hat_s b_s^T) with the
+// cumulative gate g_t and k_hat_s = k_s / g_s; with y = g_t k and z = g_t q,
+//     u = Sbar^T y + sum_s b_s (k_hat_s . y),  b = beta (v - u),
+//     o = Sbar^T z + sum_s b_s (k_hat_s . z) + b (k . q).
+// Sbar^T y and Sbar^T z are pass A of the per-step kernel with the row factors A_i y_i and
+// A_i z_i (A_i = r16_i, 1 for fp16 rows); the codes it leaves in tensor memory serve the fold
+// at the window's end, which materializes S (dequantized block, low-rank terms, gate, the new
+// token), takes the n largest |S| of the quantized rows as fp16 compensation entries, and runs
+// the per-step kernel's fit and requantize passes on the rest.
+//
+// Side block of one (slot, head): int32 count | pad to 16 B | g [d_k] fp32 |
+// (W - 1) x (k_hat [d_k] fp32, b [d_v] fp32). Two stages hold the next items' q, k, v
+// (alpha, row table), side header + g and frozen block; the low-rank terms, whose count is known
+// only once the header has landed, follow into their own buffer while pass A runs.
+// =============================================================================================
+constexpr int kMaxWin = 64;
+constexpr int kMaxCand = 256;  // candidate entries for the compensation choice
+
+// Window-only shared memory, after the per-step kernel's fixed arrays.
+constexpr uint32_t W_BAR = S_STAGE;          // full[2], tfull
+constexpr uint32_t W_Y = W_BAR + 32;         // y, z, k, g by original row
+constexpr uint32_t W_Z = W_Y + 512;
+constexpr uint32_t W_K = W_Z + 512;
+constexpr uint32_t W_GN = W_K + 512;
+constexpr uint32_t W_GNP = W_GN + 512;       // g by processing row
+constexpr uint32_t W_INV = W_GNP + 512;      // processing row of each original row
+constexpr uint32_t W_OU = W_INV + 512;       // compensation entries' contributions to u, o
+constexpr uint32_t W_OP = W_OU + 512;
+constexpr uint32_t W_LR = W_OP + 512;        // [64][2] (k_hat_s . y, k_hat_s . z)
+constexpr uint32_t W_TKEY = W_LR + 512;      // per-thread largest key
+constexpr uint32_t W_OIDX = W_TKEY + 512;    // chosen entries: flat index, position, value
+constexpr uint32_t W_OPOS = W_OIDX + 256;
+constexpr uint32_t W_OVAL = W_OPOS + 256;
+constexpr uint32_t W_MISC = W_OVAL + 256;    // [0] candidates, [1] threshold key
+constexpr uint32_t W_STAGE = W_MISC + 64;
+static_assert(W_STAGE % 16 == 0, "16-byte aligned");
+// Candidates of the compensation choice share the column-maxima buffer (used later).
+constexpr uint32_t W_CIDX = S_REDC, W_CPOS = S_REDC + 4 * kMaxCand, W_CVAL = S_REDC + 8 * kMaxCand;
+static_assert(12 * kMaxCand <= 4096, "candidates fit the column-maxima buffer");
+
+enum { F_UNDER = 2 };
+
+// Stage: header, k, q, v, (alpha), (row table), side header + g, block; two stages, then the
+// low-rank term buffer and the head table.
+struct WDPlan {
+  uint32_t esz, k_off, q_off, v_off, al_off, rt_off, sh_off, blk_off, stage, terms, tab, total;
+  __host__ __device__ WDPlan(int dk, int dv, int io, int gate, int per_row, uint32_t stage_bytes,
+                             int n_heads, int window) {
+    esz = io == 1 ? 2u : 4u;
+    k_off = (uint32_t)sizeof(StageHdr);
+    q_off = k_off + dk * esz;
+    v_off = q_off + dk * esz;
+    al_off = v_off + dv * esz;
+    rt_off = al_off + (gate == 1 ? 4u * dk : 0u);
+    sh_off = rt_off + (per_row ? 4u * dk : 0u);
+    blk_off = sh_off + 16u + 4u * dk;
+    stage = blk_off + round16(stage_bytes + kSlack);
+    terms = W_STAGE + 2u * stage;
+    tab = terms + (uint32_t)(window - 1) * 4u * (dk + dv);
+    total = tab + round16(20u * (uint32_t)n_heads);
+  }
+};
+
+// Add `add` to element (row r of the chunk, column e) of the pairs v (r, e uniform or not).
+__device__ __forceinline__ void chunk_add(float2 (&v)[8], int r, int e, float add, bool set) {
+#pragma unroll
+  for (int rr = 0; rr < 4; ++rr)
+#pragma unroll
+    for (int ee = 0; ee < 4; ++ee)
+      if (rr == r && ee == e) {
+        float& x = (rr & 1) ? v[4 * (rr >> 1) + ee].y : v[4 * (rr >> 1) + ee].x;
+        x = set ? add : x + add;
+      }
+}
+
+// One element of the tensor-memory tile, by processing row p and column j: its owner warp loads
+// the chunk, the owner lane changes the element (x += add, or x = add), the warp stores it.
+template <bool FULL>
+__device__ __forceinline__ void tile_patch(const Ctx<FULL>& c, int p, int j, float add, bool set) {
+  if (p / kRW != c.warp) return;  // warp-uniform
+  const int ch = (p % kRW) / 4;
+  uint32_t r[16];
+  float2 v[8];
+  tm_issue(c.tm + 16u * ch, r);
+  tm_take(r, v);
+  if (c.lane == j / 4) chunk_add(v, p % 4, j % 4, add, set);
+  tmem_st16x2(c.tm + 16u * ch, v);
+  tmem_wait_st();
+}
+
+// Key of an element for the compensation choice: larger |value| first; 0 = not eligible.
+__device__ __forceinline__ uint32_t wkey(float v) { return (__float_as_uint(v) & 0x7fffffffu) + 1u; }
+
+// The fold at the window's end (all threads). v of the lane's columns: cv (old c16), bv (b).
+template <int GATE, bool FULL, bool ROWS>
+__device__ __forceinline__ void window_fold(const Ctx<FULL>& c, const StepArgs& a, const uint8_t* blk,
+                                            const float* terms, int cnt, int mode,
+                                            const float4& cv, const float4& bv, uint8_t* dst,
+                                            int32_t* count) {
+  const int dk = c.dk(), dv = c.dv(), tid = c.tid, lane = c.lane;
+  const bool pivot_head = !ROWS && mode == MODE_PIVOT;
+  const int n_out = pivot_head ? 0 : a.n_outliers;
+  const uint32_t ts = (uint32_t)(dk + dv);
+  const float2 cc[4] = {dup(cv.x), dup(cv.y), dup(cv.z), dup(cv.w)};
+  const float2 bb[4] = {dup(bv.x), dup(bv.y), dup(bv.z), dup(bv.w)};
+  const float4* ak = sp<float4>(S_AK) + c.row0() / 2;
+  const float2* gnp = reinterpret_cast<const float2*>(sp<float>(W_GNP) + c.row0());
+  const uint4* rd4 = reinterpret_cast<const uint4*>(sp<uint32_t>(S_RD) + c.row0());
+  // ---- materialize S = g (x A c + sum_s k_hat_s b_s^T) + k b^T in tensor memory ----
+  sweep(c.tm, c.nch(), [&](int ch, float2 (&v)[8]) {
+    const uint4 d = rd4[ch];
+    const int orow[4] = {rd_row(d.x), rd_row(d.y), rd_row(d.z), rd_row(d.w)};
+    float2 acc[8];
+#pragma unroll
+    for (int pr = 0; pr < 2; ++pr) {
+      const float4 f = ak[2 * ch + pr];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[4 * pr + e] = __fmul2_rn(v[4 * pr + e], __fmul2_rn(lo(f), cc[e]));
+    }
+#pragma unroll 1
+    for (int s = 0; s < cnt; ++s) {
+      const float* t = terms + (size_t)s * ts;
+      const float4 b4 = c.act() ? *reinterpret_cast<const float4*>(t + dk + 4 * lane)
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float2 bs[4] = {dup(b4.x), dup(b4.y), dup(b4.z), dup(b4.w)};
+#pragma unroll
+      for (int pr = 0; pr < 2; ++pr) {
+        const float2 kh = f2(t[orow[2 * pr]], t[orow[2 * pr + 1]]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[4 * pr + e] = __ffma2_rn(kh, bs[e], acc[4 * pr + e]);
+      }
+    }
+#pragma unroll
+    for (int pr = 0; pr < 2; ++pr) {
+      const float4 f = ak[2 * ch + pr];
+      const float2 g = gnp[2 * ch + pr];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) v[4 * pr + e] = __ffma2_rn(acc[4 * pr + e], g, __fmul2_rn(hi(f), bb[e]));
+    }
+    tmem_st16x2(c.tm + 16u * ch, v);
+  });
+  tmem_wait_st();
+  __syncwarp();
+  // ---- the frozen compensation entries: S_ij += g_i value (their code is 0) ----
+  const uint8_t* ob = nullptr;
+  {
+    // byte offset of the entries: after the rows (head block = scales, rows, entries, padding)
+    uint32_t rows_end;
+    if (ROWS) {
+      rows_end = 0;
+      for (int p2 = lane; p2 < dk; p2 += 32) {
+        const uint32_t d2 = sp<uint32_t>(S_RD)[p2];
+        const uint32_t e2 = rd_off(d2) + (uint32_t)dv * (uint32_t)rd_width(d2) / 8u;
+        rows_end = rows_end > e2 ? rows_end : e2;
+      }
+      rows_end = __reduce_max_sync(0xffffffffu, rows_end);
+    } else {
+      rows_end = 2u * (dk + dv) + (uint32_t)dk * dv * (uint32_t)mode / 8u;
+    }
+    ob = blk + rows_end;
+  }
+  if (!pivot_head) {
+    for (int o = 0; o < a.n_outliers; ++o) {
+      const int idx = reinterpret_cast<const uint16_t*>(ob)[2 * o];
+      if (idx >= dk * dv) continue;
+      const float pv = __half2float(reinterpret_cast<const __half*>(ob)[2 * o + 1]);
+      const int i = idx / dv, j = idx % dv;
+      tile_patch(c, sp<int>(W_INV)[i], j, sp<float>(W_GN)[i] * pv, false);
+    }
+  }
+  // ---- the n largest |S| of the quantized rows: fp16 compensation entries ----
+  int* misc = sp<int>(W_MISC);
+  int* oidx = sp<int>(W_OIDX);
+  int* opos = sp<int>(W_OPOS);
+  float* oval = sp<float>(W_OVAL);
+  if (n_out > 0) {
+    uint32_t tmax = 0;
+    sweep(c.tm, c.nch(), [&](int ch, float2 (&v)[8]) {
+      const uint4 d = rd4[ch];
+      const uint32_t ds[4] = {d.x, d.y, d.z, d.w};
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        if (ROWS && rd_width(ds[r]) == 16) continue;
+        const float2* g = v + 4 * (r >> 1);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) tmax = max(tmax, wkey((r & 1) ? g[e].y : g[e].x));
+      }
+    });
+    sp<uint32_t>(W_TKEY)[tid] = c.act() ? tmax : 0u;
+    if (tid == 0) misc[0] = 0;
+    __syncthreads();
+    if (c.warp == 0) {  // n-th largest of the 128 thread maxima: a lower bound of the n-th element
+      uint32_t kv[kT / 32];
+#pragma unroll
+      for (int t = 0; t < kT / 32; ++t) kv[t] = sp<uint32_t>(W_TKEY)[lane * (kT / 32) + t];
+      uint32_t last = 0;
+      for (int r = 0; r < n_out; ++r) {
+        uint32_t m = 0;
+#pragma unroll
+        for (int t = 0; t < kT / 32; ++t) m = max(m, kv[t]);
+        const uint32_t wm = __reduce_max_sync(0xffffffffu, m);
+        last = wm;
+        if (wm == 0) break;
+        const uint32_t owner = __ffs(__ballot_sync(0xffffffffu, m == wm)) - 1;
+        if (lane == (int)owner) {
+          bool done = false;
+#pragma unroll
+          for (int t = 0; t < kT / 32; ++t)
+            if (!done && kv[t] == wm) {
+              kv[t] = 0;
+              done = true;
+            }
+        }
+      }
+      if (lane == 0) misc[1] = (int)(last ? last : 1u);
+    }
+    __syncthreads();
+    const uint32_t thr = (uint32_t)misc[1];
+    sweep(c.tm, c.nch(), [&](int ch, float2 (&v)[8]) {
+      const uint4 d = rd4[ch];
+      const uint32_t ds[4] = {d.x, d.y, d.z, d.w};
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        if (ROWS && rd_width(ds[r]) == 16) continue;
+        const float2* g = v + 4 * (r >> 1);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float x = (r & 1) ? g[e].y : g[e].x;
+          if (c.act() && wkey(x) >= thr) {
+            const int pos = atomicAdd(&misc[0], 1);
+            if (pos < kMaxCand) {
+              const int p = c.row0() + 4 * ch + r, j = 4 * lane + e;
+              sp<int>(W_CIDX)[pos] = rd_row(ds[r]) * dv + j;
+              sp<int>(W_CPOS)[pos] = p << 8 | j;
+              sp<float>(W_CVAL)[pos] = x;
+            }
+          }
+        }
+      }
+    });
+    __syncthreads();
+    const int nc = misc[0];
+    if (nc <= kMaxCand) {
+      if (c.warp == 0) {  // top n of the candidates by (|v| desc, flat index asc)
+        int* cidx = sp<int>(W_CIDX);
+        for (int r = 0; r < n_out; ++r) {
+          unsigned long long best = 0;
+          int bpos = -1;
+          for (int q = lane; q < nc; q += 32) {
+            const int idx = cidx[q];
+            if (idx < 0) continue;
+            const unsigned long long key =
+                ((unsigned long long)wkey(sp<float>(W_CVAL)[q]) << 32) | (0xffffffffu - (uint32_t)idx);
+            if (key > best) {
+              best = key;
+              bpos = q;
+            }
+          }
+          unsigned long long wb = best;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) {
+            const unsigned long long other = __shfl_xor_sync(0xffffffffu, wb, o);
+            wb = other > wb ? other : wb;
+          }
+          if (best == wb && bpos >= 0 && wb != 0) {
+            oidx[r] = cidx[bpos];
+            opos[r] = sp<int>(W_CPOS)[bpos];
+            oval[r] = sp<float>(W_CVAL)[bpos];
+            cidx[bpos] = -1;
+          }
+          __syncwarp();
+        }
+      }
+    } else {  // many equal values: n rounds of an exact arg-max over the tile
+      for (int r = 0; r < n_out; ++r) {
+        unsigned long long best = 0;
+        int bp = 0;
+        float bvx = 0.f;
+        sweep(c.tm, c.nch(), [&](int ch, float2 (&v)[8]) {
+          const uint4 d = rd4[ch];
+          const uint32_t ds[4] = {d.x, d.y, d.z, d.w};
+#pragma unroll
+          for (int rr = 0; rr < 4; ++rr) {
+            if (ROWS && rd_width(ds[rr]) == 16) continue;
+            const float2* g = v + 4 * (rr >> 1);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float x = (rr & 1) ? g[e].y : g[e].x;
+              const int j = 4 * lane + e, idx = rd_row(ds[rr]) * dv + j;
+              bool taken = false;
+              for (int q = 0; q < r; ++q) taken |= oidx[q] == idx;
+              if (!c.act() || taken) continue;
+              const unsigned long long key =
+                  ((unsigned long long)wkey(x) << 32) | (0xffffffffu - (uint32_t)idx);
+              if (key > best) {
+                best = key;
+                bp = (c.row0() + 4 * ch + rr) << 8 | j;
+                bvx = x;
+              }
+            }
+          }
+        });
+        unsigned long long wb = best;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          const unsigned long long other = __shfl_xor_sync(0xffffffffu, wb, o);
+          wb = other > wb ? other : wb;
+        }
+        unsigned long long* wbest = reinterpret_cast<unsigned long long*>(sp<float>(W_TKEY));
+        if (lane == 0) wbest[c.warp] = wb;
+        __syncthreads();
+        unsigned long long win = 0;
+        for (int w = 0; w < kW; ++w) win = wbest[w] > win ? wbest[w] : win;
+        if (win != 0 && best == win) {
+          oidx[r] = (int)(0xffffffffu - (uint32_t)(win & 0xffffffffu));
+          opos[r] = bp;
+          oval[r] = bvx;
+        }
+        __syncthreads();
+      }
+    }
+    __syncthreads();
+    if (tid == 0) {  // ascending flat index
+      for (int x = 1; x < n_out; ++x) {
+        const int ki = oidx[x], kp = opos[x];
+        const float kv = oval[x];
+        int y = x - 1;
+        while (y >= 0 && oidx[y] > ki) {
+          oidx[y + 1] = oidx[y];
+          opos[y + 1] = opos[y];
+          oval[y + 1] = oval[y];
+          --y;
+        }
+        oidx[y + 1] = ki;
+        opos[y + 1] = kp;
+        oval[y + 1] = kv;
+      }
+    }
+    __syncthreads();
+    for (int o = 0; o < n_out; ++o)  // out of the fit, code 0
+      tile_patch(c, opos[o] >> 8, opos[o] & 0xff, 0.f, true);
+    if (tid < n_out && __hisinf(__float2half_rn(oval[tid]))) atomicOr(&c.flags[F_RANGE], 1);
+  }
+  // ---- refit and requantize (pivot heads: round to fp16) ----
+  if (pivot_head) {
+    bool of = false;
+    sweep(c.tm, c.nch(), [&](int ch, float2 (&v)[8]) {
+      float m = 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) m = max3abs(m, v[e].x, v[e].y);
+      of |= !(m < 65520.f);
+    });
+    if (of) atomicOr(&c.flags[F_RANGE], 1);
+    __syncthreads();
+    if (c.flags[F_RANGE]) {
+      if (tid == 0) atomicOr(a.flag, SQ_FLAG_RANGE_BIT);
+    } else {
+      store_pivot(c, dst);
+    }
+    if (tid == 0) *count = 0;
+    return;
+  }
+  {  // row maxima (fp16 rows: range check)
+    float4* rtab = reinterpret_cast<float4*>(sp<float>(S_RT) + c.row0());
+    bool of = false;
+    sweep(c.tm, c.nch(), [&](int ch, float2 (&v)[8]) {
+      float rm[4];
+#pragma unroll
+      for (int pr = 0; pr < 2; ++pr) {
+        rm[2 * pr] = warp_max_nonneg(rowmax_x(v + 4 * pr));
+        rm[2 * pr + 1] = warp_max_nonneg(rowmax_y(v + 4 * pr));
+      }
+      if (lane == 0) rtab[ch] = make_float4(rm[0], rm[1], rm[2], rm[3]);
+      if (ROWS) {
+        const uint4 d = rd4[ch];
+        const uint32_t ds[4] = {d.x, d.y, d.z, d.w};
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+          if (rd_width(ds[r]) == 16 && !(rm[r] < 65520.f)) of = true;
+      }
+    });
+    if (of) atomicOr(&c.flags[F_RANGE], 1);
+    __syncwarp();
+  }
+  float r = row_scales(c, true);
+  col_pass(c, sp<float>(S_REDC));
+  __syncthreads();
+  float4 cm = max4(sp<float>(S_REDC), lane);
+  for (int f = 1; f < a.fit_iters; ++f) {
+    row_pass(c, make_float4(rcp_approx(cm.x), rcp_approx(cm.y), rcp_approx(cm.z), rcp_approx(cm.w)));
+    r = row_scales(c, false);
+    float* red = sp<float>(S_REDC) + (f & 1) * kW * kMaxD;
+    col_pass(c, red);
+    __syncthreads();
+    cm = max4(red, lane);
+  }
+  if (c.flags[F_RANGE]) {
+    if (tid == 0) {
+      atomicOr(a.flag, SQ_FLAG_RANGE_BIT);
+      *count = 0;
+    }
+    return;
+  }
+  const float4 icn = store_scales(c, dst, cm, r);
+  if (ROWS) {
+    requant_rows(c, dst, icn);
+  } else {
+    switch (mode) {
+      case 2: requant_head<2>(c, dst, icn); break;
+      case 4: requant_head<4>(c, dst, icn); break;
+      case 6: requant_head<6>(c, dst, icn); break;
+      default: requant_head<8>(c, dst, icn); break;
+    }
+  }
+  if (tid < n_out) {
+    uint8_t* o = dst + (ob - blk);
+    reinterpret_cast<uint16_t*>(o)[2 * tid] = (uint16_t)oidx[tid];
+    reinterpret_cast<__half*>(o)[2 * tid + 1] = __float2half_rn(oval[tid]);
+  }
+  if (tid == 0) *count = 0;
+}
+
+template <int GATE, int IO, bool FULL, bool ROWS>
+__global__ void __launch_bounds__(kT, 3) k_window(const StepArgs a) {
+  const WDPlan P(a.dk, a.dv, IO, GATE, ROWS, a.stage_bytes, a.H, a.window);
+  uint64_t* full = sp<uint64_t>(W_BAR);
+  uint64_t* tfull = full + 2;
+  Ctx<FULL> c;
+  c.tid = threadIdx.x;
+  c.warp = c.tid >> 5;
+  c.lane = c.tid & 31;
+  c.dk_ = a.dk;
+  c.dv_ = a.dv;
+  c.act_ = 4 * c.lane < a.dv;
+  {
+    const int rows = a.dk - c.warp * kRW;
+    c.nch_ = rows <= 0 ? 0 : (rows >= kRW ? kMaxCh : rows / 4);
+  }
+  const int H = a.H, B = a.batch, dk = c.dk(), dv = c.dv(), tid = c.tid, W = a.window;
+  const int n_items = B * H;
+  const int stride = gridDim.x;
+  const uint32_t tbytes = 4u * (uint32_t)(dk + dv);
+  float* terms = reinterpret_cast<float*>(smem + P.terms);
+
+  if (c.warp == 0) {
+    tmem_alloc(sp<uint32_t>(S_TMEM), kTmemCols);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    for (int s = 0; s < 3; ++s) mbar_init(&full[s], 1);
+    fence_mbar_init();
+  }
+  if (tid < 16) sp<int>(S_FLAGS)[tid] = 0;
+  HeadDesc* htab = reinterpret_cast<HeadDesc*>(smem + P.tab);
+  int32_t* otab = reinterpret_cast<int32_t*>(smem + P.tab + 16u * H);
+  for (int h = tid; h < H; h += kT) {
+    htab[h] = a.heads[h];
+    otab[h] = a.order[h];
+  }
+  tmem_fence_before_sync();
+  __syncthreads();
+  tmem_fence_after_sync();
+  const uint32_t tbase = *sp<uint32_t>(S_TMEM);
+  c.tm = tbase + ((uint32_t)(32 * c.warp) << 16);
+
+  Meta* meta = sp<Meta>(S_META);
+  int* flag_base = sp<int>(S_FLAGS);
+  const bool producer = c.warp == kW - 1;
+  const int first = blockIdx.x;
+  const int step_hh = stride / B, step_b = stride - step_hh * B;
+  struct Cursor {
+    int item, hh, b;
+  };
+  auto advance = [&](Cursor& k) {
+    k.item += stride;
+    k.hh += step_hh;
+    k.b += step_b;
+    if (k.b >= B) {
+      k.b -= B;
+      ++k.hh;
+    }
+  };
+  Cursor next_issue{first, first / B, first % B};
+  Cursor next_meta = next_issue;
+  auto fetch_meta = [&](Cursor& k) {
+    if (c.lane < 3 && k.item < n_items) {
+      const int io = k.b * H + otab[k.hh];
+      if (c.lane == 0) cp_async4(&meta->slot, a.slot_idx + k.b);
+      if (c.lane == 1) cp_async4(&meta->beta, a.beta + io);
+      if (c.lane == 2 && GATE == 0) cp_async4(&meta->alpha, a.alpha + io);
+      cp_async_commit();
+    }
+    advance(k);
+  };
+  auto issue = [&](Cursor& k, int s) {
+    if (c.lane < 3) cp_async_wait_all();
+    __syncwarp();
+    uint8_t* st = smem + W_STAGE + s * P.stage;
+    const int h = otab[k.hh], io = k.b * H + h;
+    const HeadDesc hd = htab[h];
+    const Meta m = *meta;
+    const bool valid = m.slot >= 0 && m.slot < a.n_slots;
+    const uint32_t kb = (uint32_t)dk * P.esz, vb = (uint32_t)dv * P.esz;
+    const uint32_t ab = GATE == 1 ? 4u * dk : 0u, rb = ROWS ? 4u * dk : 0u, shb = 16u + 4u * dk;
+    if (c.lane == 0) {
+      int* nf = flag_base + 4 * s;
+      nf[F_INPUT] = nf[F_RANGE] = nf[F_UNDER] = 0;
+      StageHdr* shdr = reinterpret_cast<StageHdr*>(st);
+      *reinterpret_cast<int4*>(shdr) = make_int4(valid, m.slot, k.b, h);
+      *(reinterpret_cast<int4*>(shdr) + 1) =
+          make_int4(__float_as_int(m.beta), __float_as_int(GATE == 0 ? m.alpha : 0.f),
+                    hd.pivot_head ? MODE_PIVOT : (int)hd.width, (int)hd.off);
+      mbar_arrive_expect_tx(&full[s], valid ? 2 * kb + vb + ab + rb + shb + hd.bytes : 0u);
+    }
+    if (valid && c.lane >= 1 && c.lane <= 7) {
+      uint8_t* dst = st;
+      const uint8_t* src = nullptr;
+      uint32_t n = 0;
+      switch (c.lane) {
+        case 1: dst += P.k_off, src = static_cast<const uint8_t*>(a.k) + (size_t)io * kb, n = kb; break;
+        case 2: dst += P.q_off, src = static_cast<const uint8_t*>(a.q) + (size_t)io * kb, n = kb; break;
+        case 3: dst += P.v_off, src = static_cast<const uint8_t*>(a.v) + (size_t)io * vb, n = vb; break;
+        case 4: dst += P.al_off, src = reinterpret_cast<const uint8_t*>(a.alpha + (size_t)io * dk), n = ab; break;
+        case 5: dst += P.rt_off, src = reinterpret_cast<const uint8_t*>(a.srows + (size_t)h * dk), n = rb; break;
+        case 6:
+          dst += P.sh_off;
+          src = a.side + (size_t)m.slot * a.side_slot_bytes + (size_t)h * a.side_head_bytes;
+          n = shb;
+          break;
+        default: dst += P.blk_off, src = a.pool + (size_t)m.slot * a.slot_bytes + hd.off, n = hd.bytes; break;
+      }
+      if (n) bulk_load(dst, src, n, &full[s]);
+    }
+    __syncwarp();
+    advance(k);
+  };
+
+  if (producer) {
+    fetch_meta(next_meta);
+    for (int s = 0; s < 2 && next_issue.item < n_items; ++s) {
+      issue(next_issue, s);
+      fetch_meta(next_meta);
+    }
+  }
+
+  int it = 0;
+  bool timed_out = false;
+  for (int item = first; item < n_items; item += stride, ++it) {
+    const int s = it & 1;
+    const uint8_t* st = smem + W_STAGE + s * P.stage;
+    const uint8_t* blk = st + P.blk_off;
+    const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&full[s], (uint32_t)(it >> 1) & 1u));
+    c.flags = flag_base + 4 * s;
+    StageHdr hdr = *reinterpret_cast<const StageHdr*>(st);
+    if (!ok) hdr.valid = 0;
+    int cnt = *reinterpret_cast<const int32_t*>(st + P.sh_off);
+    if (cnt < 0 || cnt >= W || !hdr.valid) cnt = 0;  // a closed or unreadable window restarts
+    if (tid == 0) {  // the item's low-rank terms
+      mbar_arrive_expect_tx(tfull, (uint32_t)cnt * tbytes);
+      if (cnt > 0)
+        bulk_load(terms,
+                  a.side + (size_t)hdr.slot * a.side_slot_bytes + (size_t)hdr.h * a.side_head_bytes +
+                      16u + 4u * dk,
+                  (uint32_t)cnt * tbytes, tfull);
+    }
+    const int io = hdr.b * H + hdr.h;
+    const int mode = ROWS ? MODE_ROWS : hdr.mode;
+    const bool pivot_head = !ROWS && mode == MODE_PIVOT;
+
+    // ---- setup: thread t takes processing row t, every lane its four columns ----
+    float4 cv = make_float4(1.f, 1.f, 1.f, 1.f), vv = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (hdr.valid) {
+      bool bad_in = false, under = false;
+      float kqp = 0.f;
+      const int p = tid;
+      if (p < dk) {
+        uint32_t d;
+        if (ROWS) {
+          d = reinterpret_cast<const uint32_t*>(st + P.rt_off)[p];
+        } else {
+          const uint32_t off = pivot_head ? (uint32_t)p * 2u * dv
+                                          : 2u * (dk + dv) + (uint32_t)p * dv * mode / 8u;
+          d = (uint32_t)p << 24 | off << 8 | (uint32_t)mode;
+        }
+        sp<uint32_t>(S_RD)[p] = d;
+        const int i = rd_row(d);
+        sp<int>(W_INV)[i] = p;
+        const float ki = ld_io(st + P.k_off, IO, i), qi = ld_io(st + P.q_off, IO, i);
+        const float ai = GATE == 0 ? hdr.alpha : reinterpret_cast<const float*>(st + P.al_off)[i];
+        bad_in |= !isfinite(ki) || !isfinite(qi) || !isfinite(ai);
+        const float gold = cnt > 0 ? reinterpret_cast<const float*>(st + P.sh_off + 16)[i] : 1.f;
+        const float gn = gold * ai;
+        under |= gn < 1e-30f;
+        const float yi = gn * ki, zi = gn * qi;
+        const float A = (!pivot_head && rd_width(d) != 16) ? __half2float(reinterpret_cast<const __half*>(blk)[i]) : 1.f;
+        float* gkq = sp<float>(S_GKQ) + 4 * (p >> 1) + (p & 1);
+        gkq[0] = A * yi;
+        gkq[2] = A * zi;
+        float* akp = sp<float>(S_AK) + 4 * (p >> 1) + (p & 1);
+        akp[0] = A;
+        akp[2] = ki;
+        sp<float>(W_GNP)[p] = gn;
+        sp<float>(W_Y)[i] = yi;
+        sp<float>(W_Z)[i] = zi;
+        sp<float>(W_K)[i] = ki;
+        sp<float>(W_GN)[i] = gn;
+        kqp = ki * qi;
+      }
+      kqp = warp_sum(kqp);
+      if (c.lane == 0) sp<float>(S_KQ)[c.warp] = kqp;
+      sp<float>(W_OU)[tid] = 0.f;
+      sp<float>(W_OP)[tid] = 0.f;
+      float4 icv = make_float4(1.f, 1.f, 1.f, 1.f);
+      if (c.act()) {
+        if (!pivot_head) {
+          const uint2 ch = reinterpret_cast<const uint2*>(blk + 2 * dk)[c.lane];
+          const float2 a01 = __half22float2(*reinterpret_cast<const __half2*>(&ch.x));
+          const float2 a23 = __half22float2(*reinterpret_cast<const __half2*>(&ch.y));
+          cv = make_float4(a01.x, a01.y, a23.x, a23.y);
+          if (ROWS)
+            icv = make_float4(rcp_f16val(cv.x), rcp_f16val(cv.y), rcp_f16val(cv.z), rcp_f16val(cv.w));
+        }
+        const uint8_t* vq = st + P.v_off;
+        vv = make_float4(ld_io(vq, IO, 4 * c.lane), ld_io(vq, IO, 4 * c.lane + 1),
+                         ld_io(vq, IO, 4 * c.lane + 2), ld_io(vq, IO, 4 * c.lane + 3));
+        if (c.warp == 0)
+          bad_in |= !(isfinite(vv.x) && isfinite(vv.y) && isfinite(vv.z) && isfinite(vv.w));
+      }
+      if (tid == 0) bad_in |= !isfinite(hdr.beta) || (GATE == 0 && !isfinite(hdr.alpha));
+      if (bad_in) atomicOr(&c.flags[F_INPUT], 1);
+      if (under) atomicOr(&c.flags[F_UNDER], 1);
+      __syncwarp();
+      // ---- pass A: Sbar^T y and Sbar^T z (c_j applied below); the codes stay in tensor memory
+      if (ROWS) {
+        pass_a_rows(c, blk, icv);
+      } else {
+        switch (mode) {
+          case 2: pass_a_head<2>(c, blk); break;
+          case 4: pass_a_head<4>(c, blk); break;
+          case 6: pass_a_head<6>(c, blk); break;
+          case 8: pass_a_head<8>(c, blk); break;
+          default: pass_a_head<16>(c, blk); break;
+        }
+      }
+      tmem_wait_st();
+    }
+    if (__syncthreads_or(!ok)) {  // barrier: partial sums, flags, y and z of every row
+      timed_out = true;
+      break;
+    }
+    const bool skip = !hdr.valid || c.flags[F_INPUT];
+    // frozen compensation entries' share of u and o
+    const uint8_t* ob = nullptr;
+    if (!skip && !pivot_head && a.n_outliers > 0) {
+      uint32_t rows_end;
+      if (ROWS) {
+        rows_end = 0;
+        for (int p2 = c.lane; p2 < dk; p2 += 32) {
+          const uint32_t d2 = sp<uint32_t>(S_RD)[p2];
+          const uint32_t e2 = rd_off(d2) + (uint32_t)dv * (uint32_t)rd_width(d2) / 8u;
+          rows_end = rows_end > e2 ? rows_end : e2;
+        }
+        rows_end = __reduce_max_sync(0xffffffffu, rows_end);
+      } else {
+        rows_end = 2u * (dk + dv) + (uint32_t)dk * dv * (uint32_t)mode / 8u;
+      }
+      ob = blk + rows_end;
+      if (tid < a.n_outliers) {
+        const int idx = reinterpret_cast<const uint16_t*>(ob)[2 * tid];
+        const float pv = __half2float(reinterpret_cast<const __half*>(ob)[2 * tid + 1]);
+        if (idx < dk * dv) {
+          atomicAdd(sp<float>(W_OU) + idx % dv, pv * sp<float>(W_Y)[idx / dv]);
+          atomicAdd(sp<float>(W_OP) + idx % dv, pv * sp<float>(W_Z)[idx / dv]);
+        }
+      }
+    }
+    const bool tok = __all_sync(0xffffffffu, mbar_wait_bounded(tfull, (uint32_t)it & 1u));
+    if (!skip) {  // low-rank coefficients, one term per warp at a time
+      for (int t = c.warp; t < cnt; t += kW) {
+        float dy = 0.f, dz = 0.f;
+        if (4 * c.lane < dk) {
+          const float4 kh = *reinterpret_cast<const float4*>(terms + (size_t)t * (dk + dv) + 4 * c.lane);
+          const float4 y4 = *reinterpret_cast<const float4*>(sp<float>(W_Y) + 4 * c.lane);
+          const float4 z4 = *reinterpret_cast<const float4*>(sp<float>(W_Z) + 4 * c.lane);
+          dy = __fmaf_rn(kh.x, y4.x, __fmaf_rn(kh.y, y4.y, __fmaf_rn(kh.z, y4.z, kh.w * y4.w)));
+          dz = __fmaf_rn(kh.x, z4.x, __fmaf_rn(kh.y, z4.y, __fmaf_rn(kh.z, z4.z, kh.w * z4.w)));
+        }
+        dy = warp_sum(dy);
+        dz = warp_sum(dz);
+        if (c.lane == 0) {
+          sp<float>(W_LR)[2 * t] = dy;
+          sp<float>(W_LR)[2 * t + 1] = dz;
+        }
+      }
+    }
+    if (__syncthreads_or(!tok)) {
+      timed_out = true;
+      break;
+    }
+    float* out = a.out + (size_t)io * dv;
+    if (skip) {
+      if (tid == 0) atomicOr(a.flag, hdr.valid ? SQ_FLAG_NONFINITE_BIT : SQ_FLAG_BAD_SLOT_BIT);
+      nan_out(out, dv, tid);
+    } else {
+      // ---- u, b, o for the lane's four columns ----
+      const float4 U = sum4(sp<float>(S_REDU), c.lane), Pq = sum4(sp<float>(S_REDP), c.lane);
+      float4 u = make_float4(cv.x * U.x, cv.y * U.y, cv.z * U.z, cv.w * U.w);
+      float4 pp = make_float4(cv.x * Pq.x, cv.y * Pq.y, cv.z * Pq.z, cv.w * Pq.w);
+      if (c.act()) {
+        const float4 ou = *reinterpret_cast<const float4*>(sp<float>(W_OU) + 4 * c.lane);
+        const float4 op = *reinterpret_cast<const float4*>(sp<float>(W_OP) + 4 * c.lane);
+        u = make_float4(u.x + ou.x, u.y + ou.y, u.z + ou.z, u.w + ou.w);
+        pp = make_float4(pp.x + op.x, pp.y + op.y, pp.z + op.z, pp.w + op.w);
+        for (int t = 0; t < cnt; ++t) {
+          const float4 bt = *reinterpret_cast<const float4*>(terms + (size_t)t * (dk + dv) + dk + 4 * c.lane);
+          const float ly = sp<float>(W_LR)[2 * t], lz = sp<float>(W_LR)[2 * t + 1];
+          u = make_float4(__fmaf_rn(ly, bt.x, u.x), __fmaf_rn(ly, bt.y, u.y), __fmaf_rn(ly, bt.z, u.z), __fmaf_rn(ly, bt.w, u.w));
+          pp = make_float4(__fmaf_rn(lz, bt.x, pp.x), __fmaf_rn(lz, bt.y, pp.y), __fmaf_rn(lz, bt.z, pp.z), __fmaf_rn(lz, bt.w, pp.w));
+        }
+      }
+      const float4 kq4 = *sp<float4>(S_KQ);
+      const float kqv = (kq4.x + kq4.y) + (kq4.z + kq4.w);
+      const float beta = hdr.beta;
+      const float4 bv = make_float4(beta * (vv.x - u.x), beta * (vv.y - u.y), beta * (vv.z - u.z),
+                                    beta * (vv.w - u.w));
+      uint8_t* side = a.side + (size_t)hdr.slot * a.side_slot_bytes + (size_t)hdr.h * a.side_head_bytes;
+      if (c.warp == 0 && c.act())
+        *reinterpret_cast<float4*>(out + 4 * c.lane) =
+            make_float4(__fmaf_rn(bv.x, kqv, pp.x), __fmaf_rn(bv.y, kqv, pp.y),
+                        __fmaf_rn(bv.z, kqv, pp.z), __fmaf_rn(bv.w, kqv, pp.w));
+      const bool fold = cnt + 1 >= W || c.flags[F_UNDER] != 0;
+      if (!fold) {  // append this token's factors, keep the window open
+        float* tnew = reinterpret_cast<float*>(side + 16 + 4 * dk) + (size_t)cnt * (dk + dv);
+        if (tid < dk) {
+          tnew[tid] = sp<float>(W_K)[tid] / sp<float>(W_GN)[tid];
+          reinterpret_cast<float*>(side + 16)[tid] = sp<float>(W_GN)[tid];
+        }
+        if (c.warp == 0 && c.act()) *reinterpret_cast<float4*>(tnew + dk + 4 * c.lane) = bv;
+        if (tid == 0) *reinterpret_cast<int32_t*>(side) = cnt + 1;
+      } else {  // end of the window: fold everything into the block
+        uint8_t* dst = a.pool + (size_t)hdr.slot * a.slot_bytes + hdr.off;
+        window_fold<GATE, FULL, ROWS>(c, a, blk, terms, cnt, mode, cv, bv, dst,
+                                      reinterpret_cast<int32_t*>(side));
+      }
+    }
+    __syncthreads();  // the stage and the term buffer are free
+    if (producer && next_issue.item < n_items) {
+      issue(next_issue, s);
+      fetch_meta(next_meta);
+    }
+  }
+
+  if (timed_out) {
+    if (tid == 0) atomicOr(a.flag, SQ_FLAG_TIMEOUT_BIT);
+    // let copies still in flight land before the CTA exits
+    mbar_wait_bounded(&full[it & 1], (uint32_t)(it >> 1) & 1u);
+    mbar_wait_bounded(&full[(it + 1) & 1], (uint32_t)((it + 1) >> 1) & 1u);
+    mbar_wait_bounded(tfull, (uint32_t)it & 1u);
+    if (producer && c.lane < 3) cp_async_wait_all();
+  }
+  tmem_fence_before_sync();
+  __syncthreads();
+  if (c.warp == 0) {
+    tmem_fence_after_sync();
+    tmem_dealloc(tbase, kTmemCols);
+  }
+}
+
+template <int GATE, int IO, bool FULL, bool ROWS>
+cudaError_t launch_w(const StepArgs& a, int num_sms, cudaStream_t st) {
+  auto fn = k_window<GATE, IO, FULL, ROWS>;
+  const WDPlan P(a.dk, a.dv, IO, GATE, ROWS, a.stage_bytes, a.H, a.window);
+  const uint32_t smem_bytes = P.total > 47u * 1024u ? P.total : 47u * 1024u;
+  int per_sm = 0;
+  cudaError_t e = resident_ctas(reinterpret_cast<const void*>(fn), smem_bytes, &per_sm);
+  if (e != cudaSuccess) return e;
+  if (per_sm > kMaxCtasPerSm) per_sm = kMaxCtasPerSm;
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
+  if (e != cudaSuccess) return e;
+  const int items = a.batch * a.H;
+  int grid = num_sms * per_sm;
+  if (grid > items) grid = items;
+  if (grid < 1) return cudaSuccess;
+  fn<<<grid, kT, smem_bytes, st>>>(a);
+  return cudaGetLastError();
+}
+
+template <int GATE, int IO>
+cudaError_t launch_w_shape(const StepArgs& a, int num_sms, cudaStream_t st) {
+  const bool full = a.dk == kMaxD && a.dv == kMaxD;
+  if (a.per_row)
+    return full ? launch_w<GATE, IO, true, true>(a, num_sms, st) : launch_w<GATE, IO, false, true>(a, num_sms, st);
+  return full ? launch_w<GATE, IO, true, false>(a, num_sms, st) : launch_w<GATE, IO, false, false>(a, num_sms, st);
+}
+
 }  // namespace
 
 cudaError_t launch_decode(const StepArgs& a, int gate, int io, bool want_state, int num_sms,
@@ -1043,6 +1753,14 @@ cudaError_t launch_decode(const StepArgs& a, int gate, int io, bool want_state, 
   if (gate == 1 && io == 0)
     return want_state ? launch_shape<1, 0, true>(a, num_sms, st) : launch_shape<1, 0, false>(a, num_sms, st);
   return want_state ? launch_shape<1, 1, true>(a, num_sms, st) : launch_shape<1, 1, false>(a, num_sms, st);
+}
+
+cudaError_t launch_window_step(const StepArgs& a, int gate, int io, int num_sms, cudaStream_t st) {
+  if (a.window > kMaxWin) return cudaErrorInvalidValue;
+  if (gate == 0 && io == 0) return launch_w_shape<0, 0>(a, num_sms, st);
+  if (gate == 0 && io == 1) return launch_w_shape<0, 1>(a, num_sms, st);
+  if (gate == 1 && io == 0) return launch_w_shape<1, 0>(a, num_sms, st);
+  return launch_w_shape<1, 1>(a, num_sms, st);
 }
 
 }  // namespace sq

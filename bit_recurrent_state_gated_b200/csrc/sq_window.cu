@@ -16,6 +16,7 @@
 //
 // Side block of one (slot, head): int32 count | pad to 16 B | g [d_k] fp32 |
 // W x (k_hat [d_k] fp32, b [d_v] fp32).
+#include "sq_pair.cuh"
 #include "sq_tile.cuh"
 
 namespace sq {
@@ -88,9 +89,11 @@ __device__ __forceinline__ void frozen_tile(float (&S)[kRows][4], const uint8_t*
 
 // Materialize S = g_i (Sbar_ij + sum_{s<n} khat_s[i] b_s[j]) (+ k_i b_j for a new token), then
 // choose the compensation entries, refit, requantize and store; close the window.
-__device__ __forceinline__ void flush_tile(const StepArgs& a, WSmem& sm, const uint8_t* blk,
+// kk, bcol: the new token's k and b (add_new only).
+__device__ __forceinline__ void flush_tile(const StepArgs& a, TileSmem& ts, const uint8_t* blk,
                                            const float* terms, int nterms, const float* g,
-                                           bool add_new, uint8_t* dst, const HeadDesc& hd,
+                                           bool add_new, const float* kk, const float* bcol,
+                                           uint8_t* dst, const HeadDesc& hd,
                                            const uint32_t* rows, int32_t* count) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, dk = a.dk, dv = a.dv;
   float S[kRows][4];
@@ -119,195 +122,16 @@ __device__ __forceinline__ void flush_tile(const StepArgs& a, WSmem& sm, const u
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           S[s][e] *= gi;
-          if (add_new) S[s][e] = __fmaf_rn(sm.k[i], sm.colB[4 * lane + e], S[s][e]);
+          if (add_new) S[s][e] = __fmaf_rn(kk[i], bcol[4 * lane + e], S[s][e]);
         }
       }
     }
   }
-  if (tid == 0) sm.t.misc[0] = 0;
+  if (tid == 0) ts.misc[0] = 0;
   __syncthreads();
-  const bool ok = quantize_tile(S, dst, hd, rows, a.n_outliers, a.fit_iters, warp, lane, dk, dv, sm.t);
+  const bool ok = quantize_tile(S, dst, hd, rows, a.n_outliers, a.fit_iters, warp, lane, dk, dv, ts);
   if (!ok && tid == 0) atomicOr(a.flag, SQ_FLAG_RANGE_BIT);
   if (tid == 0) *count = 0;
-}
-
-// One windowed decode step: one CTA per (request, head).
-template <int GATE, int IO>
-__global__ void __launch_bounds__(kThreads) k_window_step(const StepArgs a) {
-  extern __shared__ __align__(16) uint8_t dyn[];
-  __shared__ WSmem sm;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int dk = a.dk, dv = a.dv, H = a.H, W = a.window;
-  const int item = blockIdx.x, b = item / H, h = item % H;
-  float* out = a.out + (size_t)item * dv;
-  const int slot = a.slot_idx[b];
-  if (slot < 0 || slot >= a.n_slots) {
-    if (tid == 0) atomicOr(a.flag, SQ_FLAG_BAD_SLOT_BIT);
-    if (tid < dv) out[tid] = __int_as_float(0x7fc00000);
-    return;
-  }
-  const HeadDesc hd = a.heads[h];
-  const uint32_t* rows = a.rows + (size_t)h * dk;
-  uint8_t* dst = a.pool + (size_t)slot * a.slot_bytes + hd.off;
-  uint8_t* side = side_of(a, slot, h);
-  int32_t* count = reinterpret_cast<int32_t*>(side);
-  float* gside = reinterpret_cast<float*>(side + 16);
-  float* tside = gside + dk;  // W terms of (dk + dv) floats
-  uint8_t* blk = dyn;
-  float* terms = reinterpret_cast<float*>(dyn + round16(a.stage_bytes + kSlack));
-  const int tstride = dk + dv;
-
-  if (tid == 0) {
-    int cnt = *count;
-    if (cnt < 0 || cnt >= W) cnt = 0;  // a closed or unreadable window restarts from the block
-    sm.cnt = cnt;
-    sm.bad = 0;
-    sm.beta = a.beta[item];
-  }
-  __syncthreads();
-  const int cnt = sm.cnt;
-  copy16(blk, dst, hd.bytes, a.flag);
-  if (cnt > 0) {
-    copy16(terms, tside, (uint32_t)cnt * tstride * 4, a.flag);
-    copy16(sm.g, gside, dk * 4, a.flag);
-  }
-  bool bad = !isfinite(sm.beta);
-  if (tid < dk) {
-    const float ki = tile::ld_io(a.k, IO, item * dk + tid), qi = tile::ld_io(a.q, IO, item * dk + tid);
-    const float ai = GATE == 0 ? a.alpha[item] : a.alpha[(size_t)item * dk + tid];
-    bad |= !isfinite(ki) || !isfinite(qi) || !isfinite(ai);
-    sm.k[tid] = ki;
-    sm.q[tid] = qi;
-    sm.A[tid] = ai;  // alpha for now
-  }
-  if (tid < dv) {
-    const float vj = tile::ld_io(a.v, IO, item * dv + tid);
-    bad |= !isfinite(vj);
-    sm.v[tid] = vj;
-  }
-  if (bad) atomicOr(&sm.bad, 1);
-  __syncthreads();
-  if (sm.bad) {
-    if (tid == 0) atomicOr(a.flag, SQ_FLAG_NONFINITE_BIT);
-    if (tid < dv) out[tid] = __int_as_float(0x7fc00000);
-    return;
-  }
-  // cumulative gate, y = g k, z = g q; row factor A_i = r16_i (quantized rows) or 1
-  if (tid < dk) {
-    const float gold = cnt > 0 ? sm.g[tid] : 1.f;
-    const float gn = gold * sm.A[tid];
-    sm.g[tid] = gn;
-    sm.y[tid] = gn * sm.k[tid];
-    sm.z[tid] = gn * sm.q[tid];
-    const bool qrow = !hd.pivot_head && row_width(rows[tid]) != 16;
-    sm.A[tid] = qrow ? __half2float(reinterpret_cast<const __half*>(blk)[tid]) : 1.f;
-    if (gn < 1e-30f) atomicOr(&sm.bad, 2);  // gate underflow: fold the window in now
-  }
-  if (tid < kMaxD) {
-    float cj = 1.f;
-    if (tid < dv && !hd.pivot_head) cj = __half2float(reinterpret_cast<const __half*>(blk)[dk + tid]);
-    sm.colC[tid] = cj;
-  }
-  if (warp == 0) {
-    float kq = 0.f;
-    for (int i = lane; i < dk; i += 32) kq = __fmaf_rn(tile::ld_io(a.k, IO, item * dk + i), tile::ld_io(a.q, IO, item * dk + i), kq);
-    kq = warp_sum(kq);
-    if (lane == 0) sm.kq = kq;
-  }
-  __syncthreads();
-
-  // dense part: U_j = c_j sum_i x_ij (A_i y_i), P_j = c_j sum_i x_ij (A_i z_i)
-  {
-    float S[kRows][4];
-    unpack_tile_any(mode_of(hd), S, blk, rows, warp, lane, dk, dv);
-    float U[4] = {0.f, 0.f, 0.f, 0.f}, Pq[4] = {0.f, 0.f, 0.f, 0.f};
-    float ic[4] = {1.f, 1.f, 1.f, 1.f};
-    if (4 * lane < dv) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) ic[e] = 1.f / sm.colC[4 * lane + e];
-    }
-#pragma unroll
-    for (int s = 0; s < kRows; ++s) {
-      const int i = warp * kRows + s;
-      if (i < dk) {
-        const bool prow = !hd.pivot_head && row_width(rows[i]) == 16;
-        const float gy = sm.A[i] * sm.y[i], gz = sm.A[i] * sm.z[i];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float x = prow ? S[s][e] * ic[e] : S[s][e];
-          U[e] = __fmaf_rn(x, gy, U[e]);
-          Pq[e] = __fmaf_rn(x, gz, Pq[e]);
-        }
-      }
-    }
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      sm.t.red[warp * 2 * kMaxD + 4 * lane + e] = U[e];
-      sm.t.red[warp * 2 * kMaxD + kMaxD + 4 * lane + e] = Pq[e];
-    }
-  }
-  // low-rank part: (k_hat_s . y, k_hat_s . z) per earlier token
-  for (int t = warp; t < cnt; t += kWarps) {
-    const float* kh = terms + (size_t)t * tstride;
-    float dy = 0.f, dz = 0.f;
-    for (int i = lane; i < dk; i += 32) {
-      dy = __fmaf_rn(kh[i], sm.y[i], dy);
-      dz = __fmaf_rn(kh[i], sm.z[i], dz);
-    }
-    dy = warp_sum(dy);
-    dz = warp_sum(dz);
-    if (lane == 0) {
-      sm.lr[t][0] = dy;
-      sm.lr[t][1] = dz;
-    }
-  }
-  __syncthreads();
-  if (tid < dv) {
-    float su = 0.f, sp = 0.f;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
-      su += sm.t.red[w * 2 * kMaxD + tid];
-      sp += sm.t.red[w * 2 * kMaxD + kMaxD + tid];
-    }
-    sm.colU[tid] = sm.colC[tid] * su;
-    sm.colP[tid] = sm.colC[tid] * sp;
-  }
-  __syncthreads();
-  if (a.n_outliers > 0 && !hd.pivot_head && tid < a.n_outliers) {  // frozen fp16 entries
-    const uint8_t* o = blk + row_off(rows[dk - 1]) + (size_t)dv * row_width(rows[dk - 1]) / 8;
-    const int idx = reinterpret_cast<const uint16_t*>(o)[2 * tid];
-    const float p = __half2float(reinterpret_cast<const __half*>(o)[2 * tid + 1]);
-    if (idx < dk * dv) {
-      atomicAdd(&sm.colU[idx % dv], p * sm.y[idx / dv]);
-      atomicAdd(&sm.colP[idx % dv], p * sm.z[idx / dv]);
-    }
-  }
-  __syncthreads();
-  if (tid < dv) {
-    float u = sm.colU[tid], p = sm.colP[tid];
-    for (int t = 0; t < cnt; ++t) {
-      const float bt = terms[(size_t)t * tstride + dk + tid];
-      u = __fmaf_rn(sm.lr[t][0], bt, u);
-      p = __fmaf_rn(sm.lr[t][1], bt, p);
-    }
-    const float bj = sm.beta * (sm.v[tid] - u);
-    sm.colB[tid] = bj;
-    out[tid] = __fmaf_rn(bj, sm.kq, p);
-  }
-  __syncthreads();
-  const bool flush = cnt + 1 >= W || (sm.bad & 2);
-  if (!flush) {  // append this token's factors, keep the window open
-    float* tnew = tside + (size_t)cnt * tstride;
-    if (tid < dk) {
-      tnew[tid] = sm.k[tid] / sm.g[tid];
-      gside[tid] = sm.g[tid];
-    }
-    if (tid < dv) tnew[dk + tid] = sm.colB[tid];
-    if (tid == 0) *count = cnt + 1;
-    return;
-  }
-  // end of the window: fold everything into the block
-  flush_tile(a, sm, blk, terms, cnt, sm.g, true, dst, hd, rows, count);
 }
 
 // Fold each listed slot's open window into its block now (no-op at count 0).
@@ -334,28 +158,11 @@ __global__ void __launch_bounds__(kThreads) k_window_flush(const StepArgs a) {
   copy16(terms, side + 16 + 4 * dk, (uint32_t)cnt * (dk + dv) * 4, a.flag);
   copy16(sm.g, side + 16, dk * 4, a.flag);
   __syncthreads();
-  flush_tile(a, sm, blk, terms, cnt, sm.g, false, dst, hd, rows, count);
+  flush_tile(a, sm.t, blk, terms, cnt, sm.g, false, nullptr, nullptr, dst, hd, rows, count);
   (void)tid;
 }
 
 }  // namespace
-
-cudaError_t launch_window_step(const StepArgs& a, int gate, int io, int, cudaStream_t st) {
-  if (a.window > kMaxWindow) return cudaErrorInvalidValue;
-  const int items = a.batch * a.H;
-  if (items < 1) return cudaSuccess;
-  const uint32_t dyn = round16(a.stage_bytes + kSlack) + (uint32_t)a.window * (a.dk + a.dv) * 4;
-  auto launch = [&](auto fn) {
-    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
-    if (e != cudaSuccess) return e;
-    fn<<<items, kThreads, dyn, st>>>(a);
-    return cudaGetLastError();
-  };
-  if (gate == 0 && io == 0) return launch(k_window_step<0, 0>);
-  if (gate == 0 && io == 1) return launch(k_window_step<0, 1>);
-  if (gate == 1 && io == 0) return launch(k_window_step<1, 0>);
-  return launch(k_window_step<1, 1>);
-}
 
 cudaError_t launch_window_flush(const StepArgs& a, int, cudaStream_t st) {
   if (a.window > kMaxWindow) return cudaErrorInvalidValue;
