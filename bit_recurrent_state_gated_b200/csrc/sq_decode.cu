@@ -1074,7 +1074,8 @@ __device__ __forceinline__ void window_fold(const Ctx<FULL>& c, const StepArgs& 
       const float2 bs[4] = {dup(b4.x), dup(b4.y), dup(b4.z), dup(b4.w)};
 #pragma unroll
       for (int pr = 0; pr < 2; ++pr) {
-        const float2 kh = f2(t[orow[2 * pr]], t[orow[2 * pr + 1]]);
+        const float2 kh = ROWS ? f2(t[orow[2 * pr]], t[orow[2 * pr + 1]])
+                               : *reinterpret_cast<const float2*>(t + orow[2 * pr]);  // rows p, p+1
 #pragma unroll
         for (int e = 0; e < 4; ++e) acc[4 * pr + e] = __ffma2_rn(kh, bs[e], acc[4 * pr + e]);
       }
@@ -1516,8 +1517,8 @@ __global__ void __launch_bounds__(kT, 3) k_window(const StepArgs a) {
     const int mode = ROWS ? MODE_ROWS : hdr.mode;
     const bool pivot_head = !ROWS && mode == MODE_PIVOT;
 
-    // ---- setup: thread t takes processing row t, every lane its four columns ----
-    float4 cv = make_float4(1.f, 1.f, 1.f, 1.f), vv = make_float4(0.f, 0.f, 0.f, 0.f);
+    // ---- setup: thread t takes processing row t and value column t ----
+    float tc = 1.f, tv = 0.f;
     if (hdr.valid) {
       bool bad_in = false, under = false;
       float kqp = 0.f;
@@ -1559,21 +1560,17 @@ __global__ void __launch_bounds__(kT, 3) k_window(const StepArgs a) {
       if (c.lane == 0) sp<float>(S_KQ)[c.warp] = kqp;
       sp<float>(W_OU)[tid] = 0.f;
       sp<float>(W_OP)[tid] = 0.f;
+      if (tid < dv) {
+        if (!pivot_head) tc = __half2float(reinterpret_cast<const __half*>(blk)[dk + tid]);
+        tv = ld_io(st + P.v_off, IO, tid);
+        bad_in |= !isfinite(tv);
+      }
       float4 icv = make_float4(1.f, 1.f, 1.f, 1.f);
-      if (c.act()) {
-        if (!pivot_head) {
-          const uint2 ch = reinterpret_cast<const uint2*>(blk + 2 * dk)[c.lane];
-          const float2 a01 = __half22float2(*reinterpret_cast<const __half2*>(&ch.x));
-          const float2 a23 = __half22float2(*reinterpret_cast<const __half2*>(&ch.y));
-          cv = make_float4(a01.x, a01.y, a23.x, a23.y);
-          if (ROWS)
-            icv = make_float4(rcp_f16val(cv.x), rcp_f16val(cv.y), rcp_f16val(cv.z), rcp_f16val(cv.w));
-        }
-        const uint8_t* vq = st + P.v_off;
-        vv = make_float4(ld_io(vq, IO, 4 * c.lane), ld_io(vq, IO, 4 * c.lane + 1),
-                         ld_io(vq, IO, 4 * c.lane + 2), ld_io(vq, IO, 4 * c.lane + 3));
-        if (c.warp == 0)
-          bad_in |= !(isfinite(vv.x) && isfinite(vv.y) && isfinite(vv.z) && isfinite(vv.w));
+      if (ROWS && c.act()) {
+        const uint2 ch = reinterpret_cast<const uint2*>(blk + 2 * dk)[c.lane];
+        const float2 a01 = __half22float2(*reinterpret_cast<const __half2*>(&ch.x));
+        const float2 a23 = __half22float2(*reinterpret_cast<const __half2*>(&ch.y));
+        icv = make_float4(rcp_f16val(a01.x), rcp_f16val(a01.y), rcp_f16val(a23.x), rcp_f16val(a23.y));
       }
       if (tid == 0) bad_in |= !isfinite(hdr.beta) || (GATE == 0 && !isfinite(hdr.alpha));
       if (bad_in) atomicOr(&c.flags[F_INPUT], 1);
@@ -1598,6 +1595,13 @@ __global__ void __launch_bounds__(kT, 3) k_window(const StepArgs a) {
       break;
     }
     const bool skip = !hdr.valid || c.flags[F_INPUT];
+    float u0 = 0.f, p0 = 0.f;  // c_t (Sbar^T y)_t / c_t, (Sbar^T z)_t of column t
+    if (!skip && tid < dv) {
+      const float* ru = sp<float>(S_REDU) + tid;
+      const float* rp = sp<float>(S_REDP) + tid;
+      u0 = tc * ((ru[0] + ru[kMaxD]) + (ru[2 * kMaxD] + ru[3 * kMaxD]));
+      p0 = tc * ((rp[0] + rp[kMaxD]) + (rp[2 * kMaxD] + rp[3 * kMaxD]));
+    }
     // frozen compensation entries' share of u and o
     const uint8_t* ob = nullptr;
     if (!skip && !pivot_head && a.n_outliers > 0) {
@@ -1651,42 +1655,46 @@ __global__ void __launch_bounds__(kT, 3) k_window(const StepArgs a) {
       if (tid == 0) atomicOr(a.flag, hdr.valid ? SQ_FLAG_NONFINITE_BIT : SQ_FLAG_BAD_SLOT_BIT);
       nan_out(out, dv, tid);
     } else {
-      // ---- u, b, o for the lane's four columns ----
-      const float4 U = sum4(sp<float>(S_REDU), c.lane), Pq = sum4(sp<float>(S_REDP), c.lane);
-      float4 u = make_float4(cv.x * U.x, cv.y * U.y, cv.z * U.z, cv.w * U.w);
-      float4 pp = make_float4(cv.x * Pq.x, cv.y * Pq.y, cv.z * Pq.z, cv.w * Pq.w);
-      if (c.act()) {
-        const float4 ou = *reinterpret_cast<const float4*>(sp<float>(W_OU) + 4 * c.lane);
-        const float4 op = *reinterpret_cast<const float4*>(sp<float>(W_OP) + 4 * c.lane);
-        u = make_float4(u.x + ou.x, u.y + ou.y, u.z + ou.z, u.w + ou.w);
-        pp = make_float4(pp.x + op.x, pp.y + op.y, pp.z + op.z, pp.w + op.w);
-        for (int t = 0; t < cnt; ++t) {
-          const float4 bt = *reinterpret_cast<const float4*>(terms + (size_t)t * (dk + dv) + dk + 4 * c.lane);
-          const float ly = sp<float>(W_LR)[2 * t], lz = sp<float>(W_LR)[2 * t + 1];
-          u = make_float4(__fmaf_rn(ly, bt.x, u.x), __fmaf_rn(ly, bt.y, u.y), __fmaf_rn(ly, bt.z, u.z), __fmaf_rn(ly, bt.w, u.w));
-          pp = make_float4(__fmaf_rn(lz, bt.x, pp.x), __fmaf_rn(lz, bt.y, pp.y), __fmaf_rn(lz, bt.z, pp.z), __fmaf_rn(lz, bt.w, pp.w));
-        }
-      }
-      const float4 kq4 = *sp<float4>(S_KQ);
-      const float kqv = (kq4.x + kq4.y) + (kq4.z + kq4.w);
-      const float beta = hdr.beta;
-      const float4 bv = make_float4(beta * (vv.x - u.x), beta * (vv.y - u.y), beta * (vv.z - u.z),
-                                    beta * (vv.w - u.w));
-      uint8_t* side = a.side + (size_t)hdr.slot * a.side_slot_bytes + (size_t)hdr.h * a.side_head_bytes;
-      if (c.warp == 0 && c.act())
-        *reinterpret_cast<float4*>(out + 4 * c.lane) =
-            make_float4(__fmaf_rn(bv.x, kqv, pp.x), __fmaf_rn(bv.y, kqv, pp.y),
-                        __fmaf_rn(bv.z, kqv, pp.z), __fmaf_rn(bv.w, kqv, pp.w));
+      // ---- u, b, o of column t ----
       const bool fold = cnt + 1 >= W || c.flags[F_UNDER] != 0;
+      uint8_t* side = a.side + (size_t)hdr.slot * a.side_slot_bytes + (size_t)hdr.h * a.side_head_bytes;
+      float* tnew = reinterpret_cast<float*>(side + 16 + 4 * dk) + (size_t)cnt * (dk + dv);
+      if (tid < dv) {
+        float u = u0 + sp<float>(W_OU)[tid], pq = p0 + sp<float>(W_OP)[tid];
+        const float2* lr = reinterpret_cast<const float2*>(sp<float>(W_LR));
+        for (int t = 0; t < cnt; ++t) {
+          const float bt = terms[(size_t)t * (dk + dv) + dk + tid];
+          const float2 l = lr[t];
+          u = __fmaf_rn(l.x, bt, u);
+          pq = __fmaf_rn(l.y, bt, pq);
+        }
+        const float4 kq4 = *sp<float4>(S_KQ);
+        const float kqv = (kq4.x + kq4.y) + (kq4.z + kq4.w);
+        const float bj = hdr.beta * (tv - u);
+        out[tid] = __fmaf_rn(bj, kqv, pq);
+        if (fold)
+          sp<float>(W_OU)[tid] = bj;  // b for the fold (the column's share of u is used up)
+        else
+          tnew[dk + tid] = bj;
+      }
       if (!fold) {  // append this token's factors, keep the window open
-        float* tnew = reinterpret_cast<float*>(side + 16 + 4 * dk) + (size_t)cnt * (dk + dv);
         if (tid < dk) {
           tnew[tid] = sp<float>(W_K)[tid] / sp<float>(W_GN)[tid];
           reinterpret_cast<float*>(side + 16)[tid] = sp<float>(W_GN)[tid];
         }
-        if (c.warp == 0 && c.act()) *reinterpret_cast<float4*>(tnew + dk + 4 * c.lane) = bv;
         if (tid == 0) *reinterpret_cast<int32_t*>(side) = cnt + 1;
       } else {  // end of the window: fold everything into the block
+        __syncthreads();
+        float4 cv = make_float4(1.f, 1.f, 1.f, 1.f), bv = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (c.act()) {
+          if (!pivot_head) {
+            const uint2 ch = reinterpret_cast<const uint2*>(blk + 2 * dk)[c.lane];
+            const float2 a01 = __half22float2(*reinterpret_cast<const __half2*>(&ch.x));
+            const float2 a23 = __half22float2(*reinterpret_cast<const __half2*>(&ch.y));
+            cv = make_float4(a01.x, a01.y, a23.x, a23.y);
+          }
+          bv = *reinterpret_cast<const float4*>(sp<float>(W_OU) + 4 * c.lane);
+        }
         uint8_t* dst = a.pool + (size_t)hdr.slot * a.slot_bytes + hdr.off;
         window_fold<GATE, FULL, ROWS>(c, a, blk, terms, cnt, mode, cv, bv, dst,
                                       reinterpret_cast<int32_t*>(side));
