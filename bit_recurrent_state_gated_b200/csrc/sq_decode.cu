@@ -66,7 +66,7 @@ struct Meta {
   int32_t pad;
 };
 
-enum { F_INPUT = 0, F_RANGE = 1 };
+enum { F_INPUT = 0, F_RANGE = 1, F_BADA = 3 };
 
 // Fixed shared memory (byte offsets).
 constexpr uint32_t S_BAR = 0;                 // stage mbarrier
@@ -83,7 +83,9 @@ constexpr uint32_t S_RD = S_RT + 512;         // uint32 per row: descriptor (pro
 constexpr uint32_t S_REDU = S_RD + 512;       // [4 warps][128] partial U
 constexpr uint32_t S_REDP = S_REDU + 2048;    // [4 warps][128] partial P
 constexpr uint32_t S_REDC = S_REDP + 2048;    // [2][4 warps][128] partial column maxima
-constexpr uint32_t S_STAGE = S_REDC + 4096;   // staging buffer, then the head table
+constexpr uint32_t S_KT = S_REDC + 4096;      // float per row: k_i / A_i
+constexpr uint32_t S_TR = S_KT + 512;         // float per row: t_i, the tile holds M_ij / t_i
+constexpr uint32_t S_STAGE = S_TR + 512;      // staging buffer, then the head table
 static_assert(S_STAGE % 16 == 0 && S_GKQ % 16 == 0 && S_REDU % 16 == 0, "16-byte aligned");
 
 // Row descriptor, processing order: original row << 24 | byte offset in the block << 8 | width.
@@ -306,15 +308,21 @@ __device__ __forceinline__ void pass_a_rows(const Ctx<FULL>& c, const uint8_t* b
       make_float4(P[0].x + P[0].y, P[1].x + P[1].y, P[2].x + P[2].y, P[3].x + P[3].y);
 }
 
-// ---- pass B: M_new = x (A_i c_j) + k_i b_j in place, row maxima into S_RT -------------------
+// ---- pass B: the updated state in place, row maxima of the tile into S_RT ----------------
+// TILDE: the tile holds M_new / A_i = x_ij c_j + (k_i / A_i) b_j (one multiply and one fused
+// multiply-add per pair of elements); otherwise M_new = x_ij (A_i c_j) + k_i b_j. S_TR holds the
+// row factor t_i (A_i or 1) by which a tile row is the state; the fit and the requantization take
+// it into their row factors.
 // KIND 0: quantized head (row maxima); 1: fp16 head (fp16 range check, no maxima); 2: key-row
 // units (row maxima; range check of the fp16 rows).
-template <int KIND, bool WS, bool FULL>
+template <int KIND, bool WS, bool TILDE, bool FULL>
 __device__ __forceinline__ void pass_b(const Ctx<FULL>& c, const float4& cv, const float4& bv,
                                        float* s_new) {
   const float2 cc[4] = {dup(cv.x), dup(cv.y), dup(cv.z), dup(cv.w)};
   const float2 bb[4] = {dup(bv.x), dup(bv.y), dup(bv.z), dup(bv.w)};
   const float4* ak = sp<float4>(S_AK) + c.row0() / 2;
+  const float2* kt = reinterpret_cast<const float2*>(sp<float>(S_KT) + c.row0());
+  const float4* tr4 = reinterpret_cast<const float4*>(sp<float>(S_TR) + c.row0());
   float4* rt = reinterpret_cast<float4*>(sp<float>(S_RT) + c.row0());
   const uint4* rd4 = reinterpret_cast<const uint4*>(sp<uint32_t>(S_RD) + c.row0());
   const int dv = c.dv();
@@ -323,10 +331,16 @@ __device__ __forceinline__ void pass_b(const Ctx<FULL>& c, const float4& cv, con
     float rm[4];
 #pragma unroll
     for (int pr = 0; pr < 2; ++pr) {
-      const float4 f = ak[2 * ch + pr];
+      if (TILDE) {
+        const float2 k2 = kt[2 * ch + pr];
 #pragma unroll
-      for (int e = 0; e < 4; ++e)
-        v[4 * pr + e] = __ffma2_rn(v[4 * pr + e], __fmul2_rn(lo(f), cc[e]), __fmul2_rn(hi(f), bb[e]));
+        for (int e = 0; e < 4; ++e) v[4 * pr + e] = __ffma2_rn(k2, bb[e], __fmul2_rn(v[4 * pr + e], cc[e]));
+      } else {
+        const float4 f = ak[2 * ch + pr];
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          v[4 * pr + e] = __ffma2_rn(v[4 * pr + e], __fmul2_rn(lo(f), cc[e]), __fmul2_rn(hi(f), bb[e]));
+      }
       if (KIND != 1) {
         rm[2 * pr] = warp_max_nonneg(rowmax_x(v + 4 * pr));
         rm[2 * pr + 1] = warp_max_nonneg(rowmax_y(v + 4 * pr));
@@ -342,15 +356,19 @@ __device__ __forceinline__ void pass_b(const Ctx<FULL>& c, const float4& cv, con
     if (KIND == 2 || WS) {
       const uint4 d = rd4[ch];
       const uint32_t ds[4] = {d.x, d.y, d.z, d.w};
+      const float4 t4 = tr4[ch];
+      const float ts[4] = {t4.x, t4.y, t4.z, t4.w};
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
         const float2* g = v + 4 * (r >> 1);
+        const float t = KIND == 1 ? 1.f : ts[r];
         const float4 row = (r & 1) ? make_float4(g[0].y, g[1].y, g[2].y, g[3].y)
                                    : make_float4(g[0].x, g[1].x, g[2].x, g[3].x);
-        if (KIND == 2 && rd_width(ds[r]) == 16 && c.act())
-          of |= !(fmaxf(max3abs(row.x, row.y, row.z), fabsf(row.w)) < 65520.f);
+        if (KIND == 2 && rd_width(ds[r]) == 16 && c.act())  // |t x| < 65520
+          of |= !(t * fmaxf(max3abs(row.x, row.y, row.z), fabsf(row.w)) < 65520.f);
         if (WS && c.act())
-          *reinterpret_cast<float4*>(s_new + (size_t)rd_row(ds[r]) * dv + 4 * c.lane) = row;
+          *reinterpret_cast<float4*>(s_new + (size_t)rd_row(ds[r]) * dv + 4 * c.lane) =
+              make_float4(t * row.x, t * row.y, t * row.z, t * row.w);
       }
     }
     tmem_st16x2(c.tm + 16u * ch, v);
@@ -360,8 +378,9 @@ __device__ __forceinline__ void pass_b(const Ctx<FULL>& c, const float4& cv, con
   __syncwarp();
 }
 
-// Row scales from the row maxima in S_RT, one row per lane: r = max(m / Q, 2^-14) (at most the
-// largest fp16), w = 1 / (r Q) into S_W; fp16 rows get r = w = 0. Returns the lane's r.
+// Row scales from the row maxima in S_RT, one row per lane: m = t max |tile row|,
+// r = max(m / Q, 2^-14) (at most the largest fp16), w = 1 / (r Q); S_W gets t w, the factor of
+// the tile row in the column passes; fp16 rows get r = w = 0. Returns the lane's r.
 template <bool FULL>
 __device__ __forceinline__ float row_scales(const Ctx<FULL>& c, bool check) {
   const int p = c.row0() + c.lane;
@@ -371,10 +390,11 @@ __device__ __forceinline__ float row_scales(const Ctx<FULL>& c, bool check) {
     if (b != 16) {
       const float Q = (float)q_of_width(b);
       const float inv_q = b == 2 ? 1.0f : b == 4 ? 1.0f / 7.0f : b == 6 ? 1.0f / 31.0f : 1.0f / 127.0f;
-      const float rq = div_q(sp<float>(S_RT)[p], Q, inv_q);  // exactly m / Q
+      const float t = sp<float>(S_TR)[p];
+      const float rq = div_q(__fmul_rn(t, sp<float>(S_RT)[p]), Q, inv_q);  // exactly m / Q
       if (check && !(rq < 65520.f)) atomicOr(&c.flags[F_RANGE], 1);
       r = fminf(fmaxf(rq, kScaleFloor), 65504.f);
-      w = rcp_approx(__fmul_rn(r, Q));
+      w = __fmul_rn(t, rcp_approx(__fmul_rn(r, Q)));
     }
   }
   sp<float>(S_W)[p] = w;
@@ -444,7 +464,8 @@ __device__ __forceinline__ float4 sum4(const float* red, int lane) {
 }
 
 // ---- requantize, pack and store ----------------------------------------------------------
-// Row scales: r16_i to the block (at the original row), 1/r16_i into S_IR; column scales: c16.
+// Row scales: r16_i to the block (at the original row), t_i / r16_i into S_IR (t_i for fp16
+// rows); column scales: c16.
 // Returns the lane's correctly rounded 1/c16 of its four columns.
 template <bool FULL>
 __device__ __forceinline__ float4 store_scales(const Ctx<FULL>& c, uint8_t* dst, const float4& cm, float r) {
@@ -453,7 +474,8 @@ __device__ __forceinline__ float4 store_scales(const Ctx<FULL>& c, uint8_t* dst,
     const uint32_t d = sp<uint32_t>(S_RD)[p];
     const bool q = rd_width(d) != 16;
     const __half r16 = __float2half_rn(q ? r : 0.f);
-    sp<float>(S_IR)[p] = q ? rcp_f16val(__half2float(r16)) : 0.f;
+    const float t = sp<float>(S_TR)[p];  // fp16 rows: the factor of the stored value
+    sp<float>(S_IR)[p] = q ? __fmul_rn(t, rcp_f16val(__half2float(r16))) : t;
     reinterpret_cast<__half*>(dst)[rd_row(d)] = r16;
   }
   const __half2 c01 = __floats2half2_rn(cm.x, cm.y), c23 = __floats2half2_rn(cm.z, cm.w);
@@ -512,7 +534,9 @@ __device__ __forceinline__ void store_row_rt(int b, uint8_t* row, int lane, cons
   float s[4];
 #pragma unroll
   for (int e = 0; e < 4; ++e) s[e] = odd ? g[e].y : g[e].x;
-  if (b == 16) {
+  if (b == 16) {  // ir = t: the state value
+#pragma unroll
+    for (int e = 0; e < 4; ++e) s[e] *= ir;
     store4_f16(row, lane, s, act);
     return;
   }
@@ -681,7 +705,7 @@ __global__ void __launch_bounds__(kT, kMaxCtasPerSm) k_decode(const StepArgs a) 
     const uint32_t kb = (uint32_t)dk * P.esz, vb = (uint32_t)dv * P.esz;
     const uint32_t ab = GATE == 1 ? 4u * dk : 0u, rb = ROWS ? 4u * dk : 0u;
     if (c.lane == 0) {
-      nflags[F_INPUT] = nflags[F_RANGE] = 0;
+      nflags[F_INPUT] = nflags[F_RANGE] = nflags[F_BADA] = 0;
       StageHdr* shdr = reinterpret_cast<StageHdr*>(st);
       *reinterpret_cast<int4*>(shdr) = make_int4(valid, m.slot, k.b, h);
       *(reinterpret_cast<int4*>(shdr) + 1) =
@@ -731,7 +755,7 @@ __global__ void __launch_bounds__(kT, kMaxCtasPerSm) k_decode(const StepArgs a) 
     float4 cv = make_float4(1.f, 1.f, 1.f, 1.f), vv = make_float4(0.f, 0.f, 0.f, 0.f);
     float4 icv = make_float4(1.f, 1.f, 1.f, 1.f);
     if (hdr.valid) {
-      bool bad_in = false;
+      bool bad_in = false, bad_a = false;
       float kqp = 0.f;
       const int p = tid;
       if (p < dk) {
@@ -755,6 +779,9 @@ __global__ void __launch_bounds__(kT, kMaxCtasPerSm) k_decode(const StepArgs a) 
         float* akp = sp<float>(S_AK) + 4 * (p >> 1) + (p & 1);
         akp[0] = A;
         akp[2] = ki;
+        const bool okA = A >= 0x1p-60f && A <= 0x1p60f;  // k / A representable to full precision
+        sp<float>(S_KT)[p] = okA ? __fdiv_rn(ki, A) : 0.f;
+        bad_a = !okA;
         kqp = ki * qi;
       }
       kqp = warp_sum(kqp);
@@ -776,6 +803,7 @@ __global__ void __launch_bounds__(kT, kMaxCtasPerSm) k_decode(const StepArgs a) 
       }
       if (tid == 0) bad_in |= !isfinite(hdr.beta) || (GATE == 0 && !isfinite(hdr.alpha));
       if (bad_in) atomicOr(&c.flags[F_INPUT], 1);
+      if (bad_a) atomicOr(&c.flags[F_BADA], 1);
       __syncwarp();
       if (ROWS) {
         pass_a_rows(c, blk, icv);
@@ -831,7 +859,9 @@ __global__ void __launch_bounds__(kT, kMaxCtasPerSm) k_decode(const StepArgs a) 
     uint8_t* dst = a.pool + (size_t)hdr.slot * a.slot_bytes + hdr.off;
 
     if (!ROWS && pivot_head) {
-      pass_b<1, WS>(c, cv, bv, s_new);
+      if (tid < dk) sp<float>(S_TR)[tid] = 1.f;
+      __syncwarp();
+      pass_b<1, WS, false>(c, cv, bv, s_new);
       __syncthreads();
       if (c.flags[F_RANGE]) {
         if (tid == 0) atomicOr(a.flag, SQ_FLAG_RANGE_BIT);
@@ -842,7 +872,15 @@ __global__ void __launch_bounds__(kT, kMaxCtasPerSm) k_decode(const StepArgs a) 
     }
 
     // ---- refit: alternating row / column max-abs passes ----
-    pass_b<ROWS ? 2 : 0, WS>(c, cv, bv, s_new);
+    // head units: every row factor A_i in [2^-60, 2^60] (key-row units keep the direct form,
+    // which makes their kernels smaller)
+    const bool tilde = !ROWS && !c.flags[F_BADA];
+    if (tid < dk) sp<float>(S_TR)[tid] = tilde ? sp<float>(S_AK)[4 * (tid >> 1) + (tid & 1)] : 1.f;
+    __syncwarp();
+    if (!ROWS && tilde)
+      pass_b<ROWS ? 2 : 0, WS, !ROWS>(c, cv, bv, s_new);
+    else
+      pass_b<ROWS ? 2 : 0, WS, false>(c, cv, bv, s_new);
     float r = row_scales(c, true);
     col_pass(c, sp<float>(S_REDC));
     __syncthreads();  // barrier 2
@@ -1550,6 +1588,7 @@ __global__ void __launch_bounds__(kT, 3) k_window(const StepArgs a) {
         akp[0] = A;
         akp[2] = ki;
         sp<float>(W_GNP)[p] = gn;
+        sp<float>(S_TR)[p] = 1.f;  // the fold's tile holds the state itself
         sp<float>(W_Y)[i] = yi;
         sp<float>(W_Z)[i] = zi;
         sp<float>(W_K)[i] = ki;
