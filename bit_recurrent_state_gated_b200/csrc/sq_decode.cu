@@ -490,6 +490,24 @@ __device__ __forceinline__ float4 store_scales(const Ctx<FULL>& c, uint8_t* dst,
   return make_float4(rcp_f16val(f01.x), rcp_f16val(f01.y), rcp_f16val(f23.x), rcp_f16val(f23.y));
 }
 
+// The lane's packed codes of one row (y: floats whose low bits hold the offset codes) at p,
+// which already points at the lane's bytes of the row (2, 4, 8 bits).
+template <int B>
+__device__ __forceinline__ void store_lane(uint8_t* p, const float (&y)[4], bool act) {
+  const uint32_t y0 = __float_as_uint(y[0]), y1 = __float_as_uint(y[1]);
+  const uint32_t y2 = __float_as_uint(y[2]), y3 = __float_as_uint(y[3]);
+  if (B == 8) {
+    const uint32_t w = __byte_perm(__byte_perm(y0, y1, 0x0040u), __byte_perm(y2, y3, 0x0040u), 0x5410u);
+    if (act) *reinterpret_cast<uint32_t*>(p) = w;
+  } else if (B == 4) {
+    const uint32_t t = y0 + (y1 << 4) + (y2 << 8) + (y3 << 12);
+    if (act) *reinterpret_cast<uint16_t*>(p) = static_cast<uint16_t>(t);
+  } else {
+    const uint32_t t = y0 + (y1 << 2) + (y2 << 4) + (y3 << 6);
+    if (act) *p = static_cast<uint8_t>(t);
+  }
+}
+
 // Codes of one pair group (rows a, b of a chunk): y = fl(S fl(1/r16)) * fl(1/c16) + magic.
 __device__ __forceinline__ void quant_pair(const float2* v, float2 ir, const float2 (&ic)[4],
                                            float mgv, float ya[4], float yb[4]) {
@@ -512,18 +530,26 @@ template <int B, bool FULL>
 __device__ __forceinline__ void requant_head(const Ctx<FULL>& c, uint8_t* dst, const float4& icv) {
   const float2 ic[4] = {dup(icv.x), dup(icv.y), dup(icv.z), dup(icv.w)};
   const uint32_t rb = row_bytes_of<B>(c.dv());
-  uint8_t* row0 = dst + 2u * (c.dk() + c.dv()) + (uint32_t)c.row0() * rb;
   const float2* ir2 = reinterpret_cast<const float2*>(sp<float>(S_IR) + c.row0());
   const bool act = c.act();
   const int lane = c.lane;
+  // the lane's bytes of the warp's first row (6-bit rows: the row start; store4<6> places them)
+  uint8_t* base = dst + 2u * (c.dk() + c.dv()) + (uint32_t)c.row0() * rb +
+                  (B == 6 ? 0u : (uint32_t)lane * (B / 2));
   sweep(c.tm, c.nch(), [&](int ch, float2 (&v)[8]) {
+    uint8_t* cb = base + (uint32_t)ch * 4u * rb;
 #pragma unroll
     for (int pr = 0; pr < 2; ++pr) {
       float ya[4], yb[4];
       quant_pair(v + 4 * pr, ir2[2 * ch + pr], ic, magic_of<B>(), ya, yb);
-      uint8_t* ra = row0 + (uint32_t)(4 * ch + 2 * pr) * rb;
-      store4<B>(ra, lane, ya, act);
-      store4<B>(ra + rb, lane, yb, act);
+      uint8_t* ra = cb + (uint32_t)(2 * pr) * rb;
+      if (B == 6) {
+        store4<6>(ra, lane, ya, act);
+        store4<6>(ra + rb, lane, yb, act);
+      } else {
+        store_lane<B>(ra, ya, act);
+        store_lane<B>(ra + rb, yb, act);
+      }
     }
   });
 }
