@@ -92,10 +92,10 @@ def source_digest() -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload: str):
-    """DRAM bytes per launch of the decode kernel from the committed ncu summary, if it was
+def profiled_traffic(workload: str, kernel: str = "k_decode"):
+    """DRAM bytes per launch of the timed kernel from the committed ncu summary, if it was
     taken on the current kernel source (else None)."""
-    p = os.path.join(ROOT, "profiles", f"k_decode_{workload}.md")
+    p = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
     if not os.path.exists(p):
         return None
     digest = source_digest()
@@ -311,7 +311,7 @@ def run_ours(args, info):
     mean_launch_s = statistics.mean(kernel_ms) / 1e3
     achieved = ab["total"] * wl.batch / mean_launch_s / 1e9
     peak, peak_kind = peaks()
-    traffic = profiled_traffic(args.workload)
+    traffic = profiled_traffic(args.workload, "k_window" if wl.window > 1 else "k_decode")
     res = {
         "metric": METRIC,
         "value": total_req_steps / (dev_ms / 1e3),
@@ -340,7 +340,7 @@ def run_ours(args, info):
                      "frac": achieved / peak, "traffic": traffic,
                      "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)"
                      if peak_kind == "measured" else "fallback 6.65 TB/s",
-                     "kernel": "k_window_step" if wl.window > 1 else "k_decode",
+                     "kernel": "k_window" if wl.window > 1 else "k_decode",
                      "mean_launch_us": mean_launch_s * 1e6},
         "e2e": {"value": total_req_steps / (e2e_ms / 1e3), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
