@@ -566,16 +566,18 @@ __device__ __forceinline__ void store_row_rt(int b, uint8_t* row, int lane, cons
     store4_f16(row, lane, s, act);
     return;
   }
+  // any width 2..8: the lane's 4b bits go bytewise to byte lane * b / 2 of the row (rows of
+  // mixed-width chunks only; one code path keeps the kernel small)
   const float mg = kMagic + (float)(1 << (b - 1));
-  float y[4];
+  const uint32_t mask = (1u << b) - 1u;
+  uint32_t t = 0;
 #pragma unroll
-  for (int e = 0; e < 4; ++e) y[e] = __fmaf_rn(__fmul_rn(s[e], ir), ic[e], mg);
-  switch (b) {
-    case 2: store4<2>(row, lane, y, act); break;
-    case 4: store4<4>(row, lane, y, act); break;
-    case 6: store4<6>(row, lane, y, act); break;
-    default: store4<8>(row, lane, y, act); break;
-  }
+  for (int e = 0; e < 4; ++e)
+    t |= (__float_as_uint(__fmaf_rn(__fmul_rn(s[e], ir), ic[e], mg)) & mask) << (e * b);
+  if (!act) return;
+  uint8_t* p = row + (uint32_t)lane * (uint32_t)b / 2u;
+#pragma unroll 1
+  for (int j = 0; j < b / 2; ++j) p[j] = (uint8_t)(t >> (8 * j));
 }
 
 template <int B>
