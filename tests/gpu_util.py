@@ -115,11 +115,11 @@ def compare_codes(wl, bits, gpu_slots: np.ndarray, orc_slots: np.ndarray, what: 
     return n_mis, diff.size
 
 
-def lockstep(case: GpuCase, t: int, sample=None, want_state=True):
+def lockstep(case: GpuCase, t: int, sample=None, want_state=True, x=None):
     """One GPU step checked against the oracle started from the GPU's own pre-step bytes.
-    `sample`: request indices to check (default all)."""
+    `sample`: request indices to check (default all); `x`: inputs (default step t's)."""
     wl = case.wl
-    x = wl.step_inputs(t)
+    x = wl.step_inputs(t) if x is None else x
     pre = case.slots()
     o_gpu, s_gpu = case.step(x, want_state=want_state)
     post = case.slots()

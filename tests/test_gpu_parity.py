@@ -175,3 +175,24 @@ def test_full_size_sampled(name):
     sample = np.sort(np.random.default_rng(7).choice(wl.batch, 6, replace=False))
     for t in range(2):
         G.lockstep(case, t, sample=sample, want_state=(t == 0))
+
+
+@pytest.mark.parametrize("name", ["gdn-d128", "kda-d128", "gdn-s"])
+@pytest.mark.parametrize("want_state", [False, True])
+def test_extreme_gates(name, want_state):
+    """A gate of 0 (the old state is erased: M_new = k b^T) and a gate of 1e-30 take the
+    kernel's direct update form (the row factor A_i = alpha_i r16_i is outside [2^-60, 2^60]);
+    the other requests keep the usual form. Lockstep against the oracle."""
+    base = CASES[name]
+    wl = base.scaled(batch=3)
+    case = G.GpuCase(wl)
+    mis = tot = 0
+    for t in range(3):
+        x = wl.step_inputs(t)
+        x["alpha"] = x["alpha"].copy()
+        x["alpha"][0] = 0.0
+        x["alpha"][1] = 1e-30
+        m, n = G.lockstep(case, t, want_state=want_state, x=x)
+        mis, tot = mis + m, tot + n
+    assert mis <= max(1, 1e-4 * tot), (mis, tot)
+    assert case.pool.status() == (sq.SQ_OK, 0)
