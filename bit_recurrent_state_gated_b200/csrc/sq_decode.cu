@@ -1046,8 +1046,11 @@ constexpr uint32_t W_TKEY = W_LR + 512;      // per-thread largest key
 constexpr uint32_t W_OIDX = W_TKEY + 512;    // chosen entries: flat index, position, value
 constexpr uint32_t W_OPOS = W_OIDX + 256;
 constexpr uint32_t W_OVAL = W_OPOS + 256;
-constexpr uint32_t W_MISC = W_OVAL + 256;    // [0] candidates, [1] threshold key
-constexpr uint32_t W_STAGE = W_MISC + 64;
+constexpr uint32_t W_MISC = W_OVAL + 256;    // [0] candidates, [1] threshold key, [2] entries'
+                                             // byte offset, [4..5] items issued per stage
+constexpr uint32_t W_OE = W_MISC + 64;       // the frozen block's compensation entries:
+                                             // flat index [64] int, value [64] float
+constexpr uint32_t W_STAGE = W_OE + 512;
 static_assert(W_STAGE % 16 == 0, "16-byte aligned");
 // Candidates of the compensation choice share the column-maxima buffer (used later).
 constexpr uint32_t W_CIDX = S_REDC, W_CPOS = S_REDC + 4 * kMaxCand, W_CVAL = S_REDC + 8 * kMaxCand;
@@ -1158,28 +1161,11 @@ __device__ __forceinline__ void window_fold(const Ctx<FULL>& c, const StepArgs& 
   tmem_wait_st();
   __syncwarp();
   // ---- the frozen compensation entries: S_ij += g_i value (their code is 0) ----
-  const uint8_t* ob = nullptr;
-  {
-    // byte offset of the entries: after the rows (head block = scales, rows, entries, padding)
-    uint32_t rows_end;
-    if (ROWS) {
-      rows_end = 0;
-      for (int p2 = lane; p2 < dk; p2 += 32) {
-        const uint32_t d2 = sp<uint32_t>(S_RD)[p2];
-        const uint32_t e2 = rd_off(d2) + (uint32_t)dv * (uint32_t)rd_width(d2) / 8u;
-        rows_end = rows_end > e2 ? rows_end : e2;
-      }
-      rows_end = __reduce_max_sync(0xffffffffu, rows_end);
-    } else {
-      rows_end = 2u * (dk + dv) + (uint32_t)dk * dv * (uint32_t)mode / 8u;
-    }
-    ob = blk + rows_end;
-  }
   if (!pivot_head) {
     for (int o = 0; o < a.n_outliers; ++o) {
-      const int idx = reinterpret_cast<const uint16_t*>(ob)[2 * o];
+      const int idx = sp<int>(W_OE)[o];
       if (idx >= dk * dv) continue;
-      const float pv = __half2float(reinterpret_cast<const __half*>(ob)[2 * o + 1]);
+      const float pv = sp<float>(W_OE)[64 + o];
       const int i = idx / dv, j = idx % dv;
       tile_patch(c, sp<int>(W_INV)[i], j, sp<float>(W_GN)[i] * pv, false);
     }
@@ -1429,7 +1415,7 @@ __device__ __forceinline__ void window_fold(const Ctx<FULL>& c, const StepArgs& 
     }
   }
   if (tid < n_out) {
-    uint8_t* o = dst + (ob - blk);
+    uint8_t* o = dst + sp<int>(W_MISC)[2];
     reinterpret_cast<uint16_t*>(o)[2 * tid] = (uint16_t)oidx[tid];
     reinterpret_cast<__half*>(o)[2 * tid + 1] = __float2half_rn(oval[tid]);
   }
@@ -1508,7 +1494,7 @@ __global__ void __launch_bounds__(kT, 3) k_window(const StepArgs a) {
     }
     advance(k);
   };
-  auto issue = [&](Cursor& k, int s) {
+  auto issue = [&](Cursor& k, int s, int fslot) {
     if (c.lane < 3) cp_async_wait_all();
     __syncwarp();
     uint8_t* st = smem + W_STAGE + s * P.stage;
@@ -1519,8 +1505,9 @@ __global__ void __launch_bounds__(kT, 3) k_window(const StepArgs a) {
     const uint32_t kb = (uint32_t)dk * P.esz, vb = (uint32_t)dv * P.esz;
     const uint32_t ab = GATE == 1 ? 4u * dk : 0u, rb = ROWS ? 4u * dk : 0u, shb = 16u + 4u * dk;
     if (c.lane == 0) {
-      int* nf = flag_base + 4 * s;
+      int* nf = flag_base + 4 * fslot;
       nf[F_INPUT] = nf[F_RANGE] = nf[F_UNDER] = 0;
+      ++sp<int>(W_MISC)[4 + s];
       StageHdr* shdr = reinterpret_cast<StageHdr*>(st);
       *reinterpret_cast<int4*>(shdr) = make_int4(valid, m.slot, k.b, h);
       *(reinterpret_cast<int4*>(shdr) + 1) =
@@ -1551,10 +1538,12 @@ __global__ void __launch_bounds__(kT, 3) k_window(const StepArgs a) {
     advance(k);
   };
 
+  if (tid == 0) sp<int>(W_MISC)[4] = sp<int>(W_MISC)[5] = 0;
+  __syncthreads();
   if (producer) {
     fetch_meta(next_meta);
     for (int s = 0; s < 2 && next_issue.item < n_items; ++s) {
-      issue(next_issue, s);
+      issue(next_issue, s, s);
       fetch_meta(next_meta);
     }
   }
@@ -1566,7 +1555,7 @@ __global__ void __launch_bounds__(kT, 3) k_window(const StepArgs a) {
     const uint8_t* st = smem + W_STAGE + s * P.stage;
     const uint8_t* blk = st + P.blk_off;
     const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&full[s], (uint32_t)(it >> 1) & 1u));
-    c.flags = flag_base + 4 * s;
+    c.flags = flag_base + 4 * (it & 3);
     StageHdr hdr = *reinterpret_cast<const StageHdr*>(st);
     if (!ok) hdr.valid = 0;
     int cnt = *reinterpret_cast<const int32_t*>(st + P.sh_off);
@@ -1585,6 +1574,7 @@ __global__ void __launch_bounds__(kT, 3) k_window(const StepArgs a) {
 
     // ---- setup: thread t takes processing row t and value column t ----
     float tc = 1.f, tv = 0.f;
+    float4 cv = make_float4(1.f, 1.f, 1.f, 1.f);
     if (hdr.valid) {
       bool bad_in = false, under = false;
       float kqp = 0.f;
@@ -1632,6 +1622,21 @@ __global__ void __launch_bounds__(kT, 3) k_window(const StepArgs a) {
         tv = ld_io(st + P.v_off, IO, tid);
         bad_in |= !isfinite(tv);
       }
+      if (c.act() && !pivot_head) {  // the lane's old column scales (the fold's c)
+        const uint2 ch = reinterpret_cast<const uint2*>(blk + 2 * dk)[c.lane];
+        const float2 a01 = __half22float2(*reinterpret_cast<const __half2*>(&ch.x));
+        const float2 a23 = __half22float2(*reinterpret_cast<const __half2*>(&ch.y));
+        cv = make_float4(a01.x, a01.y, a23.x, a23.y);
+      }
+      if (!pivot_head && tid < a.n_outliers) {  // the block's compensation entries
+        const uint32_t dl = ROWS ? a.rows[(size_t)hdr.h * dk + dk - 1]
+                                 : (uint32_t)(2 * (dk + dv) + (dk - 1) * dv * mode / 8) << 8 | (uint32_t)mode;
+        const uint32_t roff = row_off(dl) + (uint32_t)dv * (uint32_t)row_width(dl) / 8u;
+        const uint8_t* o = blk + roff;
+        sp<int>(W_OE)[tid] = reinterpret_cast<const uint16_t*>(o)[2 * tid];
+        sp<float>(W_OE)[64 + tid] = __half2float(reinterpret_cast<const __half*>(o)[2 * tid + 1]);
+        if (tid == 0) sp<int>(W_MISC)[2] = (int)roff;
+      }
       float4 icv = make_float4(1.f, 1.f, 1.f, 1.f);
       if (ROWS && c.act()) {
         const uint2 ch = reinterpret_cast<const uint2*>(blk + 2 * dk)[c.lane];
@@ -1669,29 +1674,18 @@ __global__ void __launch_bounds__(kT, 3) k_window(const StepArgs a) {
       u0 = tc * ((ru[0] + ru[kMaxD]) + (ru[2 * kMaxD] + ru[3 * kMaxD]));
       p0 = tc * ((rp[0] + rp[kMaxD]) + (rp[2 * kMaxD] + rp[3 * kMaxD]));
     }
+    // the frozen block is no longer read: stage the item after next into its buffer
+    if (producer && next_issue.item < n_items) {
+      issue(next_issue, s, (it + 2) & 3);
+      fetch_meta(next_meta);
+    }
     // frozen compensation entries' share of u and o
-    const uint8_t* ob = nullptr;
-    if (!skip && !pivot_head && a.n_outliers > 0) {
-      uint32_t rows_end;
-      if (ROWS) {
-        rows_end = 0;
-        for (int p2 = c.lane; p2 < dk; p2 += 32) {
-          const uint32_t d2 = sp<uint32_t>(S_RD)[p2];
-          const uint32_t e2 = rd_off(d2) + (uint32_t)dv * (uint32_t)rd_width(d2) / 8u;
-          rows_end = rows_end > e2 ? rows_end : e2;
-        }
-        rows_end = __reduce_max_sync(0xffffffffu, rows_end);
-      } else {
-        rows_end = 2u * (dk + dv) + (uint32_t)dk * dv * (uint32_t)mode / 8u;
-      }
-      ob = blk + rows_end;
-      if (tid < a.n_outliers) {
-        const int idx = reinterpret_cast<const uint16_t*>(ob)[2 * tid];
-        const float pv = __half2float(reinterpret_cast<const __half*>(ob)[2 * tid + 1]);
-        if (idx < dk * dv) {
-          atomicAdd(sp<float>(W_OU) + idx % dv, pv * sp<float>(W_Y)[idx / dv]);
-          atomicAdd(sp<float>(W_OP) + idx % dv, pv * sp<float>(W_Z)[idx / dv]);
-        }
+    if (!skip && !pivot_head && tid < a.n_outliers) {
+      const int idx = sp<int>(W_OE)[tid];
+      const float pv = sp<float>(W_OE)[64 + tid];
+      if (idx < dk * dv) {
+        atomicAdd(sp<float>(W_OU) + idx % dv, pv * sp<float>(W_Y)[idx / dv]);
+        atomicAdd(sp<float>(W_OP) + idx % dv, pv * sp<float>(W_Z)[idx / dv]);
       }
     }
     const bool tok = __all_sync(0xffffffffu, mbar_wait_bounded(tfull, (uint32_t)it & 1u));
@@ -1752,33 +1746,25 @@ __global__ void __launch_bounds__(kT, 3) k_window(const StepArgs a) {
         if (tid == 0) *reinterpret_cast<int32_t*>(side) = cnt + 1;
       } else {  // end of the window: fold everything into the block
         __syncthreads();
-        float4 cv = make_float4(1.f, 1.f, 1.f, 1.f), bv = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (c.act()) {
-          if (!pivot_head) {
-            const uint2 ch = reinterpret_cast<const uint2*>(blk + 2 * dk)[c.lane];
-            const float2 a01 = __half22float2(*reinterpret_cast<const __half2*>(&ch.x));
-            const float2 a23 = __half22float2(*reinterpret_cast<const __half2*>(&ch.y));
-            cv = make_float4(a01.x, a01.y, a23.x, a23.y);
-          }
-          bv = *reinterpret_cast<const float4*>(sp<float>(W_OU) + 4 * c.lane);
-        }
+        float4 bv = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (c.act()) bv = *reinterpret_cast<const float4*>(sp<float>(W_OU) + 4 * c.lane);
         uint8_t* dst = a.pool + (size_t)hdr.slot * a.slot_bytes + hdr.off;
         window_fold<GATE, FULL, ROWS>(c, a, blk, terms, cnt, mode, cv, bv, dst,
                                       reinterpret_cast<int32_t*>(side));
       }
     }
-    __syncthreads();  // the stage and the term buffer are free
-    if (producer && next_issue.item < n_items) {
-      issue(next_issue, s);
-      fetch_meta(next_meta);
-    }
+    __syncthreads();  // the term buffer and this item's shared arrays are free
   }
 
   if (timed_out) {
     if (tid == 0) atomicOr(a.flag, SQ_FLAG_TIMEOUT_BIT);
-    // let copies still in flight land before the CTA exits
-    mbar_wait_bounded(&full[it & 1], (uint32_t)(it >> 1) & 1u);
-    mbar_wait_bounded(&full[(it + 1) & 1], (uint32_t)((it + 1) >> 1) & 1u);
+    // let copies still in flight land before the CTA exits: stage s has received
+    // W_MISC[4 + s] copies, of which the items before `it` consumed (it + 1 - s) / 2
+    __syncthreads();
+    for (int s2 = 0; s2 < 2; ++s2) {
+      const int issued = sp<int>(W_MISC)[4 + s2], used = (it + 1 - s2) / 2;
+      for (int u = used; u < issued; ++u) mbar_wait_bounded(&full[s2], (uint32_t)u & 1u);
+    }
     mbar_wait_bounded(tfull, (uint32_t)it & 1u);
     if (producer && c.lane < 3) cp_async_wait_all();
   }
