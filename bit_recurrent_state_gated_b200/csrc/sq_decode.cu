@@ -1054,7 +1054,8 @@ constexpr uint32_t W_STAGE = W_OE + 512;
 static_assert(W_STAGE % 16 == 0, "16-byte aligned");
 // Candidates of the compensation choice share the column-maxima buffer (used later).
 constexpr uint32_t W_CIDX = S_REDC, W_CPOS = S_REDC + 4 * kMaxCand, W_CVAL = S_REDC + 8 * kMaxCand;
-static_assert(12 * kMaxCand <= 4096, "candidates fit the column-maxima buffer");
+constexpr uint32_t W_CSEL = S_REDC + 12 * kMaxCand;  // the chosen n in key order: idx, pos, value
+static_assert(12 * kMaxCand + 3 * 64 * 4 <= 4096, "candidates fit the column-maxima buffer");
 
 enum { F_UNDER = 2 };
 
@@ -1093,17 +1094,27 @@ __device__ __forceinline__ void chunk_add(float2 (&v)[8], int r, int e, float ad
 
 // One element of the tensor-memory tile, by processing row p and column j: its owner warp loads
 // the chunk, the owner lane changes the element (x += add, or x = add), the warp stores it.
+// Returns the element's new value to the owner lane (0 elsewhere).
 template <bool FULL>
-__device__ __forceinline__ void tile_patch(const Ctx<FULL>& c, int p, int j, float add, bool set) {
-  if (p / kRW != c.warp) return;  // warp-uniform
+__device__ __forceinline__ float tile_patch(const Ctx<FULL>& c, int p, int j, float add, bool set) {
+  if (p / kRW != c.warp) return 0.f;  // warp-uniform
   const int ch = (p % kRW) / 4;
   uint32_t r[16];
   float2 v[8];
   tm_issue(c.tm + 16u * ch, r);
   tm_take(r, v);
-  if (c.lane == j / 4) chunk_add(v, p % 4, j % 4, add, set);
+  float nv = 0.f;
+  if (c.lane == j / 4) {
+    chunk_add(v, p % 4, j % 4, add, set);
+#pragma unroll
+    for (int rr = 0; rr < 4; ++rr)
+#pragma unroll
+      for (int ee = 0; ee < 4; ++ee)
+        if (rr == p % 4 && ee == j % 4) nv = (rr & 1) ? v[4 * (rr >> 1) + ee].y : v[4 * (rr >> 1) + ee].x;
+  }
   tmem_st16x2(c.tm + 16u * ch, v);
   tmem_wait_st();
+  return nv;
 }
 
 // Key of an element for the compensation choice: larger |value| first; 0 = not eligible.
@@ -1124,7 +1135,9 @@ __device__ __forceinline__ void window_fold(const Ctx<FULL>& c, const StepArgs& 
   const float4* ak = sp<float4>(S_AK) + c.row0() / 2;
   const float2* gnp = reinterpret_cast<const float2*>(sp<float>(W_GNP) + c.row0());
   const uint4* rd4 = reinterpret_cast<const uint4*>(sp<uint32_t>(S_RD) + c.row0());
-  // ---- materialize S = g (x A c + sum_s k_hat_s b_s^T) + k b^T in tensor memory ----
+  // ---- materialize S = g (x A c + sum_s k_hat_s b_s^T) + k b^T in tensor memory; the thread's
+  // largest |S| over the rows eligible for compensation entries ----
+  float tmaxf = 0.f;
   sweep(c.tm, c.nch(), [&](int ch, float2 (&v)[8]) {
     const uint4 d = rd4[ch];
     const int orow[4] = {rd_row(d.x), rd_row(d.y), rd_row(d.z), rd_row(d.w)};
@@ -1156,6 +1169,14 @@ __device__ __forceinline__ void window_fold(const Ctx<FULL>& c, const StepArgs& 
 #pragma unroll
       for (int e = 0; e < 4; ++e) v[4 * pr + e] = __ffma2_rn(acc[4 * pr + e], g, __fmul2_rn(hi(f), bb[e]));
     }
+    if (ROWS) {  // fp16 rows are not eligible for the compensation entries
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+        if (rd_width((&d.x)[r]) != 16) tmaxf = fmaxf(tmaxf, (r & 1) ? rowmax_y(v + 4 * (r >> 1)) : rowmax_x(v + 4 * (r >> 1)));
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) tmaxf = max3abs(tmaxf, v[e].x, v[e].y);
+    }
     tmem_st16x2(c.tm + 16u * ch, v);
   });
   tmem_wait_st();
@@ -1167,7 +1188,7 @@ __device__ __forceinline__ void window_fold(const Ctx<FULL>& c, const StepArgs& 
       if (idx >= dk * dv) continue;
       const float pv = sp<float>(W_OE)[64 + o];
       const int i = idx / dv, j = idx % dv;
-      tile_patch(c, sp<int>(W_INV)[i], j, sp<float>(W_GN)[i] * pv, false);
+      tmaxf = fmaxf(tmaxf, fabsf(tile_patch(c, sp<int>(W_INV)[i], j, sp<float>(W_GN)[i] * pv, false)));
     }
   }
   // ---- the n largest |S| of the quantized rows: fp16 compensation entries ----
@@ -1176,19 +1197,7 @@ __device__ __forceinline__ void window_fold(const Ctx<FULL>& c, const StepArgs& 
   int* opos = sp<int>(W_OPOS);
   float* oval = sp<float>(W_OVAL);
   if (n_out > 0) {
-    uint32_t tmax = 0;
-    sweep(c.tm, c.nch(), [&](int ch, float2 (&v)[8]) {
-      const uint4 d = rd4[ch];
-      const uint32_t ds[4] = {d.x, d.y, d.z, d.w};
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        if (ROWS && rd_width(ds[r]) == 16) continue;
-        const float2* g = v + 4 * (r >> 1);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) tmax = max(tmax, wkey((r & 1) ? g[e].y : g[e].x));
-      }
-    });
-    sp<uint32_t>(W_TKEY)[tid] = c.act() ? tmax : 0u;
+    sp<uint32_t>(W_TKEY)[tid] = c.act() ? wkey(tmaxf) : 0u;
     if (tid == 0) misc[0] = 0;
     __syncthreads();
     if (c.warp == 0) {  // n-th largest of the 128 thread maxima: a lower bound of the n-th element
@@ -1219,6 +1228,10 @@ __device__ __forceinline__ void window_fold(const Ctx<FULL>& c, const StepArgs& 
     __syncthreads();
     const uint32_t thr = (uint32_t)misc[1];
     sweep(c.tm, c.nch(), [&](int ch, float2 (&v)[8]) {
+      float cmx = 0.f;  // the chunk's largest |S| (all rows) bounds its candidates
+#pragma unroll
+      for (int e = 0; e < 8; ++e) cmx = max3abs(cmx, v[e].x, v[e].y);
+      if (!c.act() || wkey(cmx) < thr) return;
       const uint4 d = rd4[ch];
       const uint32_t ds[4] = {d.x, d.y, d.z, d.w};
 #pragma unroll
@@ -1243,35 +1256,33 @@ __device__ __forceinline__ void window_fold(const Ctx<FULL>& c, const StepArgs& 
     __syncthreads();
     const int nc = misc[0];
     if (nc <= kMaxCand) {
-      if (c.warp == 0) {  // top n of the candidates by (|v| desc, flat index asc)
-        int* cidx = sp<int>(W_CIDX);
-        for (int r = 0; r < n_out; ++r) {
-          unsigned long long best = 0;
-          int bpos = -1;
-          for (int q = lane; q < nc; q += 32) {
-            const int idx = cidx[q];
-            if (idx < 0) continue;
-            const unsigned long long key =
-                ((unsigned long long)wkey(sp<float>(W_CVAL)[q]) << 32) | (0xffffffffu - (uint32_t)idx);
-            if (key > best) {
-              best = key;
-              bpos = q;
-            }
-          }
-          unsigned long long wb = best;
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) {
-            const unsigned long long other = __shfl_xor_sync(0xffffffffu, wb, o);
-            wb = other > wb ? other : wb;
-          }
-          if (best == wb && bpos >= 0 && wb != 0) {
-            oidx[r] = cidx[bpos];
-            opos[r] = sp<int>(W_CPOS)[bpos];
-            oval[r] = sp<float>(W_CVAL)[bpos];
-            cidx[bpos] = -1;
-          }
-          __syncwarp();
+      // rank of each candidate by (|v| desc, flat index asc); the first n go to the stage
+      // arrays in that order, then to oidx/opos/oval in ascending flat index
+      int* sidx = sp<int>(W_CSEL);
+      int* spos = sidx + 64;
+      float* sval = reinterpret_cast<float*>(sidx + 128);
+      for (int q = tid; q < nc; q += kT) {
+        const int qi = sp<int>(W_CIDX)[q];
+        const uint32_t qk = wkey(sp<float>(W_CVAL)[q]);
+        int rank = 0;
+        for (int u = 0; u < nc; ++u) {
+          const uint32_t uk = wkey(sp<float>(W_CVAL)[u]);
+          rank += (uk > qk || (uk == qk && sp<int>(W_CIDX)[u] < qi)) ? 1 : 0;
         }
+        if (rank < n_out) {
+          sidx[rank] = qi;
+          spos[rank] = sp<int>(W_CPOS)[q];
+          sval[rank] = sp<float>(W_CVAL)[q];
+        }
+      }
+      __syncthreads();
+      if (tid < n_out) {
+        const int mi = sidx[tid];
+        int rank = 0;
+        for (int u = 0; u < n_out; ++u) rank += sidx[u] < mi ? 1 : 0;
+        oidx[rank] = mi;
+        opos[rank] = spos[tid];
+        oval[rank] = sval[tid];
       }
     } else {  // many equal values: n rounds of an exact arg-max over the tile
       for (int r = 0; r < n_out; ++r) {
@@ -1322,7 +1333,7 @@ __device__ __forceinline__ void window_fold(const Ctx<FULL>& c, const StepArgs& 
       }
     }
     __syncthreads();
-    if (tid == 0) {  // ascending flat index
+    if (nc > kMaxCand && tid == 0) {  // fallback path: ascending flat index
       for (int x = 1; x < n_out; ++x) {
         const int ki = oidx[x], kp = opos[x];
         const float kv = oval[x];
