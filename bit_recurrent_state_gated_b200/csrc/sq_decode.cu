@@ -1154,12 +1154,15 @@ __device__ __forceinline__ void window_fold(const Ctx<FULL>& c, const StepArgs& 
       const float4 b4 = c.act() ? *reinterpret_cast<const float4*>(t + dk + 4 * lane)
                                 : make_float4(0.f, 0.f, 0.f, 0.f);
       const float2 bs[4] = {dup(b4.x), dup(b4.y), dup(b4.z), dup(b4.w)};
+      float4 k4;  // k_hat of the chunk's four rows (head units: rows 4ch..4ch+3, one load)
+      if (ROWS)
+        k4 = make_float4(t[orow[0]], t[orow[1]], t[orow[2]], t[orow[3]]);
+      else
+        k4 = *reinterpret_cast<const float4*>(t + orow[0]);
 #pragma unroll
-      for (int pr = 0; pr < 2; ++pr) {
-        const float2 kh = ROWS ? f2(t[orow[2 * pr]], t[orow[2 * pr + 1]])
-                               : *reinterpret_cast<const float2*>(t + orow[2 * pr]);  // rows p, p+1
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[4 * pr + e] = __ffma2_rn(kh, bs[e], acc[4 * pr + e]);
+      for (int e = 0; e < 4; ++e) {
+        acc[e] = __ffma2_rn(lo(k4), bs[e], acc[e]);
+        acc[4 + e] = __ffma2_rn(hi(k4), bs[e], acc[4 + e]);
       }
     }
 #pragma unroll
