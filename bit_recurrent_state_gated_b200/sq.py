@@ -85,6 +85,7 @@ def lib() -> C.CDLL:
         "sq_window_flush": [P, P, I32, P],
         "sq_pool_status": [P, C.POINTER(I32)],
         "sq_debug_decode_step_fp32": [P, P, I32, P, P, P, P, P, P, P, P],
+        "sq_allocate_bits": [I32, P, P, C.c_float, I32, P, P],
     }
     for name, args in sigs.items():
         fn = getattr(L, name)
@@ -167,6 +168,20 @@ def sq_debug_decode_step_fp32(pool: int, slot_idx: int, batch: int, q: int, k: i
 
 def sq_window_flush(pool: int, slot_idx: int, n: int, stream: int) -> None:
     _chk(lib().sq_window_flush(pool, slot_idx, n, stream), "sq_window_flush")
+
+
+def sq_allocate_bits(variance, lifetime, avg_bits: float, n_pivots: int = 0):
+    """Unit widths under an average budget (host): returns (bits_map, pivot_mask) uint8."""
+    var = np.ascontiguousarray(np.asarray(variance, dtype=np.float32))
+    life = np.ascontiguousarray(np.asarray(lifetime, dtype=np.float32))
+    if var.shape != life.shape or var.ndim != 1:
+        raise ValueError("variance and lifetime must be 1-D arrays of one length")
+    bits = np.zeros(var.size, dtype=np.uint8)
+    piv = np.zeros(var.size, dtype=np.uint8)
+    _chk(lib().sq_allocate_bits(var.size, var.ctypes.data, life.ctypes.data, float(avg_bits),
+                                int(n_pivots), bits.ctypes.data, piv.ctypes.data),
+         "sq_allocate_bits")
+    return bits, piv
 
 
 def sq_pool_status(pool: int) -> tuple[int, int]:

@@ -167,6 +167,28 @@ SQ_API sq_status sq_window_flush(sq_pool* pool, const int32_t* slot_idx, int32_t
  * Returns SQ_OK, SQ_ERR_DEVICE_FLAG or SQ_ERR_TIMEOUT. */
 SQ_API sq_status sq_pool_status(sq_pool* pool, int32_t* device_flag);
 
+/*
+ * Offline width allocation (host; no device work). [SQ-E] lifetime-aware allocation paragraph:
+ * under a fixed average bit budget, units whose error is large and long-lived get more bits,
+ * chosen from a score combining each unit's reconstruction distortion with the mean lifetime of
+ * its memory; a few high-risk units stay FP16 (pivots). The Block-GTQ page's greedy rule (the
+ * next bits to the unit whose error they reduce most) decides the widths.
+ *   n_units           units (heads for SQ_UNIT_HEAD, H * d_k key rows for SQ_UNIT_KEY_ROW)
+ *   variance (host)   [n_units] variance of the unit's state entries, >= 0, finite
+ *   lifetime (host)   [n_units] mean lifetime of the unit's memory in steps, >= 0, finite
+ *                     (1 / (1 - mean gate) for a gate keeping a fraction alpha per step)
+ *   avg_bits          mean width of the non-pivot units, in [2, 8]
+ *   n_pivots          units kept FP16: the largest risks lifetime * variance (ties: lower index)
+ *   bits_map (host)   [n_units] out: 2, 4, 6, 8, or 16 for a pivot (the pool's bits_map)
+ *   pivot_mask (host) [n_units] out, may be NULL: 1 where bits_map is 16
+ * Non-pivot units start at 2 bits and receive floor((avg_bits - 2) n' / 2) steps of 2 bits
+ * (n' non-pivot units; widths at most 8), each to the unit with the largest reduction of
+ * lifetime * variance * 2^(-2 b) (ties: lower index); this minimizes the total of that score.
+ * Returns SQ_ERR_INVALID_ARG for a bad count, budget or statistic (nothing written). */
+SQ_API sq_status sq_allocate_bits(int32_t n_units, const float* variance, const float* lifetime,
+                                  float avg_bits, int32_t n_pivots, uint8_t* bits_map,
+                                  uint8_t* pivot_mask);
+
 /* Text of a status code (static storage). */
 SQ_API const char* sq_status_string(sq_status status);
 

@@ -76,6 +76,7 @@ def lib():
             "orc_decode_step": [P, P, P, P, C.c_int, P, P, P, P, P, P, P, C.c_int],
             "orc_window_step": [P, P, P, P, C.c_int, P, P, P, P, P, P, P, P, C.c_int],
             "orc_window_flush": [P, P, P, P, C.c_int, P, P, C.c_int],
+            "orc_allocate_bits": [C.c_int, P, P, C.c_double, C.c_int, P, P],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -273,3 +274,14 @@ class Pool:
         _chk(lib().orc_window_flush(C.byref(self._lay), _p(self.bits), _p(self.data), _p(si),
                                     si.size, _p(self.wstate), _p(self.count),
                                     threads or default_threads()), "window_flush")
+
+
+def allocate_bits(variance, lifetime, avg_bits: float, n_pivots: int = 0):
+    """The optimal widths under the budget (exact dynamic program): (bits, objective)."""
+    var = np.ascontiguousarray(np.asarray(variance, dtype=np.float64))
+    life = np.ascontiguousarray(np.asarray(lifetime, dtype=np.float64))
+    bits = np.zeros(var.size, dtype=np.uint8)
+    obj = C.c_double(0.0)
+    _chk(lib().orc_allocate_bits(var.size, _p(var), _p(life), float(avg_bits), int(n_pivots),
+                                 _p(bits), C.byref(obj)), "allocate_bits")
+    return bits, float(obj.value)

@@ -697,3 +697,91 @@ int orc_window_flush(const orc_layout* L, const uint8_t* bits, uint8_t* pool,
   free(off);
   return err;
 }
+
+/* ----------------------------------------------------------------------------------------
+ * Offline width allocation. [SQ-E] lifetime-aware allocation paragraph: under a fixed average
+ * bit budget, units whose error is large and long-lived get more bits, from a score that
+ * combines the unit's reconstruction distortion with the mean lifetime of its memory; a few
+ * high-risk units stay FP16 (pivots).
+ *
+ * Reading (the pages give no formula): unit u has risk R_u = lifetime_u * variance_u and, at b
+ * bits, score R_u 2^(-2b) (a uniform b-bit quantizer's distortion scales as variance 2^(-2b)).
+ * The n_pivots largest risks (ties: lower index) are pivots (width 16). The other n' units take
+ * widths in {2, 4, 6, 8} with exactly K = floor((avg_bits - 2) n' / 2) steps of 2 bits above 2,
+ * chosen to MINIMIZE sum_u R_u 2^(-2 b_u). This function solves that problem exactly by dynamic
+ * programming over (unit, steps used) -- the plain definition of the optimum, independent of
+ * any greedy rule. Returns the minimum in *objective (sum over non-pivot units).
+ * ---------------------------------------------------------------------------------------- */
+int orc_allocate_bits(int n, const double* variance, const double* lifetime, double avg_bits,
+                      int n_pivots, uint8_t* bits_out, double* objective) {
+  if (n < 1 || n_pivots < 0 || n_pivots >= n || !(avg_bits >= 2.0 && avg_bits <= 8.0))
+    return ORC_ERR_ARG;
+  double* R = (double*)malloc(sizeof(double) * n);
+  int* is_piv = (int*)calloc((size_t)n, sizeof(int));
+  if (!R || !is_piv) {
+    free(R);
+    free(is_piv);
+    return ORC_ERR_ARG;
+  }
+  for (int u = 0; u < n; ++u) R[u] = variance[u] * lifetime[u];
+  for (int p = 0; p < n_pivots; ++p) {  // the largest remaining risk, lowest index on ties
+    int best = -1;
+    for (int u = 0; u < n; ++u)
+      if (!is_piv[u] && (best < 0 || R[u] > R[best])) best = u;
+    is_piv[best] = 1;
+  }
+  const int nq = n - n_pivots;
+  long K = (long)floor((avg_bits - 2.0) * nq / 2.0 + 1e-9);
+  if (K < 0) K = 0;
+  if (K > 3L * nq) K = 3L * nq;
+  /* f[k] = least score of the units seen so far using exactly k steps; choice[u][k] = steps
+   * given to unit u in that optimum */
+  double* f = (double*)malloc(sizeof(double) * (K + 1));
+  double* g = (double*)malloc(sizeof(double) * (K + 1));
+  uint8_t* choice = (uint8_t*)malloc((size_t)n * (K + 1));
+  if (!f || !g || !choice) {
+    free(R);
+    free(is_piv);
+    free(f);
+    free(g);
+    free(choice);
+    return ORC_ERR_ARG;
+  }
+  for (long k = 0; k <= K; ++k) f[k] = k == 0 ? 0.0 : INFINITY;
+  for (int u = 0; u < n; ++u) {
+    if (is_piv[u]) continue;
+    for (long k = 0; k <= K; ++k) {
+      double best = INFINITY;
+      int bl = 0;
+      for (int l = 0; l <= 3 && l <= k; ++l) {
+        const double v = f[k - l] + R[u] * pow(2.0, -2.0 * (2 + 2 * l));
+        if (v < best) {
+          best = v;
+          bl = l;
+        }
+      }
+      g[k] = best;
+      choice[(size_t)u * (K + 1) + k] = (uint8_t)bl;
+    }
+    double* t = f;
+    f = g;
+    g = t;
+  }
+  if (objective) *objective = f[K];
+  long k = K;
+  for (int u = n - 1; u >= 0; --u) {
+    if (is_piv[u]) {
+      bits_out[u] = 16;
+      continue;
+    }
+    const int l = choice[(size_t)u * (K + 1) + k];
+    bits_out[u] = (uint8_t)(2 + 2 * l);
+    k -= l;
+  }
+  free(R);
+  free(is_piv);
+  free(f);
+  free(g);
+  free(choice);
+  return ORC_OK;
+}

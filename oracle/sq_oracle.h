@@ -74,6 +74,10 @@ int orc_window_flush(const orc_layout* L, const uint8_t* bits, uint8_t* pool,
                      const int32_t* slot_idx, int n, double* wstate, int32_t* count,
                      int n_threads);
 
+/* ---- offline width allocation (exact optimum by dynamic programming) ---- */
+int orc_allocate_bits(int n, const double* variance, const double* lifetime, double avg_bits,
+                      int n_pivots, uint8_t* bits_out, double* objective);
+
 #ifdef __cplusplus
 }
 #endif
