@@ -6,8 +6,11 @@ dual-axis refit, requantize and repack in place) over one batch of synthetic req
 default workload is the GDN-style layer: 64 requests x 32 heads, d_k = d_v = 128, per-head
 widths {4, 6, 8} (mean 6) plus 2 fp16 pivot heads, bf16 q/k/v.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload gdn|kda|pool]
-                    [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W]
+                    [--workload gdn|kda|pool|window|chunk] [--impl ours|reference]
+
+The chunk workload is the GDN layer advanced 8 tokens per call (sq_decode_chunk); one step is
+one call, and it counts batch x 8 request-steps.
 
 Prints one JSON line (rank 0). Multi-GPU: launched by torchrun, one process per GPU, each rank
 decoding its own requests (weak scaling, no collective on the data path); times are device
@@ -45,7 +48,7 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="gdn", choices=["tiny", "gdn", "kda", "pool", "window"])
+    ap.add_argument("--workload", default="gdn", choices=["tiny", "gdn", "kda", "pool", "window", "chunk"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
@@ -58,11 +61,14 @@ def algorithmic_bytes(wl: W.Workload, slot_bytes: int) -> dict:
     """Bytes one request-step must move: the packed state (codes, scales, fp16 units) read and
     written, q/k/v read, alpha/beta read, o written, the slot index read. Windowed layouts read
     the frozen block every token and write it once per window; their low-rank side state
-    (the cumulative gate and one (k_hat, b) pair per token, fp32) is counted as `side`."""
+    (the cumulative gate and one (k_hat, b) pair per token, fp32) is counted as `side`. A chunk
+    of T tokens reads and writes the packed state once: 1/T of it per request-step."""
     esz = 2 if wl.io_dtype == W.IO_BF16 else 4
     H, dk, dv = wl.n_heads, wl.d_k, wl.d_v
     io = H * (2 * dk + dv) * esz + H * wl.alpha_width * 4 + H * 4 + H * dv * 4 + 4
-    if wl.window <= 1:
+    if wl.tokens > 1:
+        state, side = 2 * slot_bytes / wl.tokens, 0
+    elif wl.window <= 1:
         state, side = 2 * slot_bytes, 0
     else:
         Wn = wl.window
@@ -183,14 +189,16 @@ def oracle_rate(wl: W.Workload, seconds: float, t0: int = 0):
     import oracle
     threads = oracle.default_threads()
     n_req = max(1, min(wl.batch, threads))
-    lay = oracle.Layout(wl.n_heads, wl.d_k, wl.d_v, wl.unit, wl.gate, wl.fit_iters, wl.window,
+    # a chunk of T tokens is the windowed oracle with W = T (requantized after the T-th token)
+    window = wl.tokens if wl.tokens > 1 else wl.window
+    lay = oracle.Layout(wl.n_heads, wl.d_k, wl.d_v, wl.unit, wl.gate, wl.fit_iters, window,
                         wl.n_outliers)
     pool = oracle.Pool(lay, wl.bits(), n_req)
-    step = pool.window_step if wl.window > 1 else pool.decode_step
+    step = pool.window_step if window > 1 else pool.decode_step
     si = np.arange(n_req, dtype=np.int32)
     pool.quantize(si, wl.initial_state(wl.slot_idx()[:n_req]))
     sets = []
-    for t in range(t0, t0 + 4):
+    for t in range(t0, t0 + max(4, wl.tokens)):
         x = wl.step_inputs(t)
         sets.append({k: np.ascontiguousarray(v[:n_req]) for k, v in x.items()})
     done, busy, n = 0, 0.0, 0
@@ -224,10 +232,11 @@ def run_ours(args, info):
     for c in range(0, wl.batch, 64):  # initial states, quantized on the GPU in chunks
         S0 = torch.from_numpy(wl.initial_state(si_np[c:c + 64])).cuda()
         pool.quantize(si[c:c + 64], S0)
+    T = wl.tokens
     n_sets = max(1, min(args.steps + args.warmup, 8))
     sets_host, sets_dev = [], []
     for t in range(n_sets):
-        x = wl.step_inputs(t)
+        x = wl.chunk_inputs(t * T, T) if T > 1 else wl.step_inputs(t)
         if wl.io_dtype == W.IO_BF16:
             qkv = [torch.from_numpy(x[n + "_bf16"]).view(torch.bfloat16) for n in "qkv"]
         else:
@@ -236,7 +245,8 @@ def run_ours(args, info):
                                                torch.from_numpy(x["beta"])]]
         sets_host.append(host)
         sets_dev.append([a.cuda() for a in host])
-    out = torch.empty((wl.batch, wl.n_heads, wl.d_v), dtype=torch.float32, device="cuda")
+    out = torch.empty((wl.batch, wl.n_heads) + ((T,) if T > 1 else ()) + (wl.d_v,),
+                      dtype=torch.float32, device="cuda")
     out_host = torch.empty(out.shape, dtype=torch.float32).pin_memory()
     flush_buf = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
     sink = torch.empty(1, dtype=torch.float32, device="cuda")
@@ -251,10 +261,16 @@ def run_ours(args, info):
     stream = torch.cuda.current_stream()
     st_handle = stream.cuda_stream
 
+    def call(q, k, v, a, b):
+        if T > 1:
+            sq.sq_decode_chunk(pool.handle, si.data_ptr(), wl.batch, T, q, k, v, a, b,
+                               out.data_ptr(), st_handle)
+        else:
+            sq.sq_decode_step(pool.handle, si.data_ptr(), wl.batch, q, k, v, a, b,
+                              out.data_ptr(), st_handle)
+
     def step(t):
-        q, k, v, a, b = sets_dev[t % n_sets]
-        sq.sq_decode_step(pool.handle, si.data_ptr(), wl.batch, q.data_ptr(), k.data_ptr(),
-                          v.data_ptr(), a.data_ptr(), b.data_ptr(), out.data_ptr(), st_handle)
+        call(*(x.data_ptr() for x in sets_dev[t % n_sets]))
 
     log(f"pool ready: {wl.slots} slots x {pool.slot_bytes} B; warm-up")
     for t in range(args.warmup):
@@ -305,8 +321,7 @@ def run_ours(args, info):
         flush.zero_()
         ev2[t][0].record(stream)
         d_packed.copy_(packed_host[(args.warmup + t) % n_sets], non_blocking=True)
-        sq.sq_decode_step(pool.handle, si.data_ptr(), wl.batch, qp, kp, vp, ap, bp,
-                          out.data_ptr(), st_handle)
+        call(qp, kp, vp, ap, bp)
         out_host.copy_(out, non_blocking=True)
         ev2[t][1].record(stream)
     torch.cuda.synchronize()
@@ -318,12 +333,13 @@ def run_ours(args, info):
     h2d = total
     d2h = out_host.numel() * out_host.element_size()
 
-    total_req_steps = wl.batch * args.steps * info.world
+    total_req_steps = wl.batch * T * args.steps * info.world
     ab = algorithmic_bytes(wl, pool.slot_bytes)
     mean_launch_s = statistics.mean(kernel_ms) / 1e3
-    achieved = ab["total"] * wl.batch / mean_launch_s / 1e9
+    achieved = ab["total"] * wl.batch * T / mean_launch_s / 1e9
     peak, peak_kind = peaks()
-    traffic = profiled_traffic(args.workload, "k_window" if wl.window > 1 else "k_decode")
+    kernel = "k_chunk" if T > 1 else "k_window" if wl.window > 1 else "k_decode"
+    traffic = profiled_traffic(args.workload, kernel)
     res = {
         "metric": METRIC,
         "value": total_req_steps / (dev_ms / 1e3),
@@ -345,6 +361,7 @@ def run_ours(args, info):
             "state_bytes_per_request": pool.slot_bytes,
             "algorithmic_bytes_per_request_step": ab["total"],
             "window": wl.window, "compensation_entries_per_head": wl.n_outliers,
+            "tokens_per_call": T,
             "l2": "flushed before every timed step (write, then read, 256 MB)",
             "parallelism": f"dp{info.world} (requests partitioned, no collective)",
         },
@@ -352,7 +369,7 @@ def run_ours(args, info):
                      "frac": achieved / peak, "traffic": traffic,
                      "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)"
                      if peak_kind == "measured" else "fallback 6.65 TB/s",
-                     "kernel": "k_window" if wl.window > 1 else "k_decode",
+                     "kernel": kernel,
                      "mean_launch_us": mean_launch_s * 1e6},
         "e2e": {"value": total_req_steps / (e2e_ms / 1e3), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},

@@ -333,6 +333,21 @@ sq_status sq_decode_step(sq_pool* pool, const int32_t* slot_idx, int32_t batch, 
   return cuda_status(sq::launch_decode(a, pool->L.gate, pool->L.io_dtype, false, pool->num_sms, st));
 }
 
+sq_status sq_decode_chunk(sq_pool* pool, const int32_t* slot_idx, int32_t batch, int32_t n_tokens,
+                          const void* q, const void* k, const void* v, const float* alpha,
+                          const float* beta, float* out, void* stream) {
+  if (!pool || n_tokens < 1 || n_tokens > sq::kMaxChunkTokens) return SQ_ERR_INVALID_ARG;
+  sq_status s = check_step(pool, slot_idx, batch, q, k, v, alpha, beta, out);
+  if (s != SQ_OK || batch == 0) return s;
+  if (pool->L.window > 1) return SQ_ERR_UNSUPPORTED;
+  sq::StepArgs a = step_args(pool, slot_idx, batch, q, k, v, alpha, beta, out, nullptr);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (n_tokens == 1)  // one token is the decode step
+    return cuda_status(sq::launch_decode(a, pool->L.gate, pool->L.io_dtype, false, pool->num_sms, st));
+  a.n_tok = n_tokens;
+  return cuda_status(sq::launch_chunk(a, pool->L.gate, pool->L.io_dtype, pool->num_sms, st));
+}
+
 sq_status sq_debug_decode_step_fp32(sq_pool* pool, const int32_t* slot_idx, int32_t batch,
                                     const void* q, const void* k, const void* v,
                                     const float* alpha, const float* beta, float* out,

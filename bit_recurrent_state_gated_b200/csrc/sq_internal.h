@@ -53,6 +53,7 @@ struct StepArgs {
   uint8_t* side;          // side region base (n_slots * side_slot_bytes)
   int64_t side_slot_bytes, side_head_bytes;
   int32_t window, n_outliers;
+  int32_t n_tok;  // tokens of a chunk (sq_decode_chunk)
 };
 
 struct QuantArgs {
@@ -80,5 +81,7 @@ cudaError_t launch_dequantize(const QuantArgs& a, cudaStream_t st);
 cudaError_t launch_window_step(const StepArgs& a, int gate, int io, int num_sms,
                                cudaStream_t st);
 cudaError_t launch_window_flush(const StepArgs& a, int num_sms, cudaStream_t st);
+cudaError_t launch_chunk(const StepArgs& a, int gate, int io, int num_sms, cudaStream_t st);
+constexpr int kMaxChunkTokens = 16;
 
 }  // namespace sq

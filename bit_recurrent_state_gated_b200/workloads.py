@@ -59,6 +59,7 @@ class Workload:
     fit_iters: int = 2
     window: int = 1
     n_outliers: int = 0
+    tokens: int = 1                # tokens per call (> 1: the multi-token chunk step)
     init_std: float = 0.1
     notes: str = field(default="", compare=False)
 
@@ -147,9 +148,17 @@ class Workload:
                      v=np.ascontiguousarray(v))
         return d
 
+    def chunk_inputs(self, t0: int, n: int) -> dict:
+        """Steps t0 .. t0+n-1 of step_inputs stacked on a token axis after the head axis:
+        q, k [B][H][n][d_k], v [B][H][n][d_v], alpha [B][H][n] or [B][H][n][d_k], beta
+        [B][H][n] (and the bf16 patterns with bf16 I/O)."""
+        steps = [self.step_inputs(t0 + t) for t in range(n)]
+        return {name: np.ascontiguousarray(np.stack([x[name] for x in steps], axis=2))
+                for name in steps[0]}
 
-# The five workloads: a tiny oracle check, a GDN layer, a KDA layer, a serving pool and the
-# windowed variant. Bit mixes: averages are over the non-pivot units.
+
+# The workloads: a tiny oracle check, a GDN layer, a KDA layer, a serving pool, the windowed
+# variant and the GDN layer in 8-token chunks. Bit mixes: averages are over the non-pivot units.
 WORKLOADS = {
     "tiny": Workload(
         name="tiny", batch=2, n_heads=2, d_k=16, d_v=16, steps=8, gate=GATE_SCALAR,
@@ -175,6 +184,12 @@ WORKLOADS = {
         unit=UNIT_HEAD, io_dtype=IO_BF16, mix=((8, 32),), n_pivots=0, seed=4, alpha_min=0.9,
         window=16, n_outliers=8,
         notes="8-bit, requantize every 16 tokens, top-8 |S| per head kept fp16"),
+    "chunk": Workload(
+        name="chunk", batch=64, n_heads=32, d_k=128, d_v=128, steps=256, gate=GATE_SCALAR,
+        unit=UNIT_HEAD, io_dtype=IO_BF16, mix=((4, 10), (6, 10), (8, 10)), n_pivots=2, seed=1,
+        alpha_min=0.9, tokens=8,
+        notes="the GDN layer advanced 8 tokens per call (prefill / speculative decode chunk), "
+              "requantized once per call"),
 }
 
 

@@ -159,6 +159,25 @@ SQ_API sq_status sq_decode_step(sq_pool* pool, const int32_t* slot_idx, int32_t 
                          const void* k, const void* v, const float* alpha, const float* beta,
                          float* out, void* stream);
 
+/*
+ * n_tokens consecutive tokens of each request in one call (prefill, or speculative decode into a
+ * quantized state): the state is read from the pool once, advanced through the tokens in fp32 on
+ * chip, and refit and requantized once, after the last token. Each token's update and output
+ * are those of sq_decode_step ([SQ-E] gated Delta rule paragraph); quantizing only after the
+ * last of them is the window-end requantization of [LQ-N] with W = n_tokens and no
+ * compensation entries. n_tokens == 1 is sq_decode_step. Pools with window == 1 only
+ * (SQ_ERR_UNSUPPORTED otherwise); 1 <= n_tokens <= 16 (SQ_ERR_INVALID_ARG otherwise).
+ *   slot_idx (device) int32 [batch]
+ *   q, k (device) [batch][n_heads][n_tokens][d_k], v (device) [batch][n_heads][n_tokens][d_v]
+ *   alpha (device) fp32 [batch][n_heads][n_tokens] or [batch][n_heads][n_tokens][d_k]
+ *   beta (device) fp32 [batch][n_heads][n_tokens]
+ *   out (device) fp32 [batch][n_heads][n_tokens][d_v]
+ * Pointers 16-byte aligned. A request with a non-finite input is skipped (its slot unchanged,
+ * its outputs NaN, SQ_FLAG_NONFINITE set). */
+SQ_API sq_status sq_decode_chunk(sq_pool* pool, const int32_t* slot_idx, int32_t batch,
+                                 int32_t n_tokens, const void* q, const void* k, const void* v,
+                                 const float* alpha, const float* beta, float* out, void* stream);
+
 /* Windowed pools: fold each listed slot's open window into its quantized block now and close
  * the window (no-op for a closed window). slot_idx (device) [n]. */
 SQ_API sq_status sq_window_flush(sq_pool* pool, const int32_t* slot_idx, int32_t n, void* stream);
