@@ -10,7 +10,9 @@ widths {4, 6, 8} (mean 6) plus 2 fp16 pivot heads, bf16 q/k/v.
                     [--workload gdn|kda|pool|window|chunk] [--impl ours|reference]
 
 The chunk workload is the GDN layer advanced 8 tokens per call (sq_decode_chunk); one step is
-one call, and it counts batch x 8 request-steps.
+one call, and it counts batch x 8 request-steps. The split workload is the GDN layer through
+sq_decode_step_split (update on one stream, refit + requantize on a second); a step ends when
+both streams are done.
 
 Prints one JSON line (rank 0). Multi-GPU: launched by torchrun, one process per GPU, each rank
 decoding its own requests (weak scaling, no collective on the data path); times are device
@@ -48,7 +50,8 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="gdn", choices=["tiny", "gdn", "kda", "pool", "window", "chunk"])
+    ap.add_argument("--workload", default="gdn", choices=["tiny", "gdn", "kda", "pool", "window", "chunk",
+                                                     "split"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
@@ -261,8 +264,19 @@ def run_ours(args, info):
     stream = torch.cuda.current_stream()
     st_handle = stream.cuda_stream
 
+    staging = side = None
+    if wl.side_stream:
+        staging = torch.empty((wl.batch, wl.n_heads, wl.d_k, wl.d_v), dtype=torch.float32,
+                              device="cuda")
+        side = torch.cuda.Stream()
+
     def call(q, k, v, a, b):
-        if T > 1:
+        if wl.side_stream:
+            sq.sq_decode_step_split(pool.handle, si.data_ptr(), wl.batch, q, k, v, a, b,
+                                    out.data_ptr(), staging.data_ptr(), st_handle,
+                                    side.cuda_stream)
+            stream.wait_stream(side)  # the step ends when the requantization has
+        elif T > 1:
             sq.sq_decode_chunk(pool.handle, si.data_ptr(), wl.batch, T, q, k, v, a, b,
                                out.data_ptr(), st_handle)
         else:
@@ -338,7 +352,8 @@ def run_ours(args, info):
     mean_launch_s = statistics.mean(kernel_ms) / 1e3
     achieved = ab["total"] * wl.batch * T / mean_launch_s / 1e9
     peak, peak_kind = peaks()
-    kernel = "k_chunk" if T > 1 else "k_window" if wl.window > 1 else "k_decode"
+    kernel = ("k_chunk" if T > 1 else "k_window" if wl.window > 1 else
+              "k_decode (update only) + k_quantize" if wl.side_stream else "k_decode")
     traffic = profiled_traffic(args.workload, kernel)
     res = {
         "metric": METRIC,
@@ -362,6 +377,7 @@ def run_ours(args, info):
             "algorithmic_bytes_per_request_step": ab["total"],
             "window": wl.window, "compensation_entries_per_head": wl.n_outliers,
             "tokens_per_call": T,
+            "side_stream_split": wl.side_stream,
             "l2": "flushed before every timed step (write, then read, 256 MB)",
             "parallelism": f"dp{info.world} (requests partitioned, no collective)",
         },
@@ -373,7 +389,7 @@ def run_ours(args, info):
                      "mean_launch_us": mean_launch_s * 1e6},
         "e2e": {"value": total_req_steps / (e2e_ms / 1e3), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps * (2 if wl.side_stream else 1),
         "clocks": clocks.summary(),
     }
     log("end-to-end region done")

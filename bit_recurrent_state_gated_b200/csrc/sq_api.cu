@@ -26,6 +26,9 @@ struct sq_pool {
   int32_t* d_order = nullptr;
   int32_t* d_flag = nullptr;
   int device = 0, num_sms = 0;
+  // side-stream split: the last split's requantization, which later calls on the pool wait for
+  cudaEvent_t ev_update = nullptr, ev_side = nullptr;
+  bool side_pending = false;
 };
 
 namespace {
@@ -201,6 +204,11 @@ sq::QuantArgs quant_args(sq_pool* p, const int32_t* slot_idx, int32_t n, const f
   return a;
 }
 
+// Order `st` after the requantization a side-stream split left running on the pool.
+cudaError_t after_side(sq_pool* p, cudaStream_t st) {
+  return p->side_pending ? cudaStreamWaitEvent(st, p->ev_side, 0) : cudaSuccess;
+}
+
 sq_status check_step(sq_pool* p, const int32_t* slot_idx, int32_t batch, const void* q,
                      const void* k, const void* v, const float* alpha, const float* beta,
                      const float* out) {
@@ -289,6 +297,8 @@ sq_status sq_state_pool_destroy(sq_pool* pool) {
   cudaFree(pool->d_srows);
   cudaFree(pool->d_flag);
   cudaFree(pool->d_order);
+  if (pool->ev_update) cudaEventDestroy(pool->ev_update);
+  if (pool->ev_side) cudaEventDestroy(pool->ev_side);
   delete pool;
   return SQ_OK;
 }
@@ -309,7 +319,9 @@ sq_status sq_quantize_fp32_state(sq_pool* pool, const int32_t* slot_idx, int32_t
   if (n == 0) return SQ_OK;
   if (!slot_idx || !S || !aligned(slot_idx, 4) || !aligned(S, 16)) return SQ_ERR_INVALID_ARG;
   const sq::QuantArgs a = quant_args(pool, slot_idx, n, S, nullptr);
-  return cuda_status(sq::launch_quantize(a, static_cast<cudaStream_t>(stream)));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaError_t e = after_side(pool, st)) return cuda_status(e);
+  return cuda_status(sq::launch_quantize(a, st));
 }
 
 sq_status sq_dequantize_state(sq_pool* pool, const int32_t* slot_idx, int32_t n, float* S_out,
@@ -318,7 +330,9 @@ sq_status sq_dequantize_state(sq_pool* pool, const int32_t* slot_idx, int32_t n,
   if (n == 0) return SQ_OK;
   if (!slot_idx || !S_out || !aligned(slot_idx, 4) || !aligned(S_out, 16)) return SQ_ERR_INVALID_ARG;
   const sq::QuantArgs a = quant_args(pool, slot_idx, n, nullptr, S_out);
-  return cuda_status(sq::launch_dequantize(a, static_cast<cudaStream_t>(stream)));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaError_t e = after_side(pool, st)) return cuda_status(e);
+  return cuda_status(sq::launch_dequantize(a, st));
 }
 
 sq_status sq_decode_step(sq_pool* pool, const int32_t* slot_idx, int32_t batch, const void* q,
@@ -328,6 +342,7 @@ sq_status sq_decode_step(sq_pool* pool, const int32_t* slot_idx, int32_t batch, 
   if (s != SQ_OK || batch == 0) return s;
   const sq::StepArgs a = step_args(pool, slot_idx, batch, q, k, v, alpha, beta, out, nullptr);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaError_t e = after_side(pool, st)) return cuda_status(e);
   if (pool->L.window > 1)
     return cuda_status(sq::launch_window_step(a, pool->L.gate, pool->L.io_dtype, pool->num_sms, st));
   return cuda_status(sq::launch_decode(a, pool->L.gate, pool->L.io_dtype, false, pool->num_sms, st));
@@ -342,6 +357,7 @@ sq_status sq_decode_chunk(sq_pool* pool, const int32_t* slot_idx, int32_t batch,
   if (pool->L.window > 1) return SQ_ERR_UNSUPPORTED;
   sq::StepArgs a = step_args(pool, slot_idx, batch, q, k, v, alpha, beta, out, nullptr);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaError_t e = after_side(pool, st)) return cuda_status(e);
   if (n_tokens == 1)  // one token is the decode step
     return cuda_status(sq::launch_decode(a, pool->L.gate, pool->L.io_dtype, false, pool->num_sms, st));
   a.n_tok = n_tokens;
@@ -357,8 +373,37 @@ sq_status sq_debug_decode_step_fp32(sq_pool* pool, const int32_t* slot_idx, int3
   if (pool->L.window > 1) return SQ_ERR_UNSUPPORTED;
   if (!s_new || !aligned(s_new, 16)) return SQ_ERR_INVALID_ARG;
   const sq::StepArgs a = step_args(pool, slot_idx, batch, q, k, v, alpha, beta, out, s_new);
-  return cuda_status(sq::launch_decode(a, pool->L.gate, pool->L.io_dtype, true, pool->num_sms,
-                                       static_cast<cudaStream_t>(stream)));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaError_t e = after_side(pool, st)) return cuda_status(e);
+  return cuda_status(sq::launch_decode(a, pool->L.gate, pool->L.io_dtype, true, pool->num_sms, st));
+}
+
+sq_status sq_decode_step_split(sq_pool* pool, const int32_t* slot_idx, int32_t batch,
+                               const void* q, const void* k, const void* v, const float* alpha,
+                               const float* beta, float* out, float* staging, void* stream,
+                               void* side_stream) {
+  sq_status s = check_step(pool, slot_idx, batch, q, k, v, alpha, beta, out);
+  if (s != SQ_OK || batch == 0) return s;
+  if (pool->L.window > 1) return SQ_ERR_UNSUPPORTED;
+  if (!staging || !aligned(staging, 16)) return SQ_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream), side = static_cast<cudaStream_t>(side_stream);
+  cudaError_t e = cudaSuccess;
+  if (!pool->ev_update) {
+    if ((e = cudaEventCreateWithFlags(&pool->ev_update, cudaEventDisableTiming)) ||
+        (e = cudaEventCreateWithFlags(&pool->ev_side, cudaEventDisableTiming)))
+      return cuda_status(e);
+  }
+  if ((e = after_side(pool, st))) return cuda_status(e);
+  sq::StepArgs a = step_args(pool, slot_idx, batch, q, k, v, alpha, beta, out, staging);
+  a.update_only = 1;
+  if ((e = sq::launch_decode(a, pool->L.gate, pool->L.io_dtype, true, pool->num_sms, st)) ||
+      (e = cudaEventRecord(pool->ev_update, st)) || (e = cudaStreamWaitEvent(side, pool->ev_update, 0)))
+    return cuda_status(e);
+  const sq::QuantArgs qa = quant_args(pool, slot_idx, batch, staging, nullptr);
+  if ((e = sq::launch_quantize(qa, side)) || (e = cudaEventRecord(pool->ev_side, side)))
+    return cuda_status(e);
+  pool->side_pending = true;
+  return SQ_OK;
 }
 
 sq_status sq_window_flush(sq_pool* pool, const int32_t* slot_idx, int32_t n, void* stream) {

@@ -863,6 +863,7 @@ __global__ void __launch_bounds__(kT, kMaxCtasPerSm) k_decode(const StepArgs a) 
     }
     if (c.flags[F_INPUT]) {  // non-finite input somewhere in the item: skip it
       if (tid == 0) atomicOr(a.flag, SQ_FLAG_NONFINITE_BIT);
+      if (WS && a.update_only && tid == 0) a.s_new[(size_t)io * dk * dv] = __int_as_float(0x7fc00000);
       nan_out(out, dv, tid);
       continue;
     }
@@ -891,6 +892,7 @@ __global__ void __launch_bounds__(kT, kMaxCtasPerSm) k_decode(const StepArgs a) 
       __syncwarp();
       pass_b<1, WS, false>(c, cv, bv, s_new);
       __syncthreads();
+      if (WS && a.update_only) continue;
       if (c.flags[F_RANGE]) {
         if (tid == 0) atomicOr(a.flag, SQ_FLAG_RANGE_BIT);
         continue;
@@ -909,6 +911,10 @@ __global__ void __launch_bounds__(kT, kMaxCtasPerSm) k_decode(const StepArgs a) 
       pass_b<ROWS ? 2 : 0, WS, !ROWS>(c, cv, bv, s_new);
     else
       pass_b<ROWS ? 2 : 0, WS, false>(c, cv, bv, s_new);
+    if (WS && a.update_only) {  // the refit and requantization run elsewhere
+      __syncthreads();
+      continue;
+    }
     float r = row_scales(c, true);
     col_pass(c, sp<float>(S_REDC));
     __syncthreads();  // barrier 2
@@ -1948,8 +1954,9 @@ __device__ __forceinline__ void rebase_tile(const Ctx<FULL>& c, const float* ter
   __syncwarp();
 }
 
+// Head units: 3 CTAs per SM (shared memory holds a pivot head's 32 KB tile); key-row units: 4.
 template <int GATE, int IO, bool FULL, bool ROWS>
-__global__ void __launch_bounds__(kT, 2) k_chunk(const StepArgs a) {
+__global__ void __launch_bounds__(kT, ROWS ? 4 : 3) k_chunk(const StepArgs a) {
   const int T = a.n_tok;
   const CPlan P(a.dk, a.dv, IO, GATE, ROWS, a.stage_bytes, a.H, T);
   uint64_t* full = sp<uint64_t>(W_BAR);

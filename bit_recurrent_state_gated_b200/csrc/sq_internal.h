@@ -54,6 +54,8 @@ struct StepArgs {
   int64_t side_slot_bytes, side_head_bytes;
   int32_t window, n_outliers;
   int32_t n_tok;  // tokens of a chunk (sq_decode_chunk)
+  int32_t update_only;  // with s_new: write the updated fp32 state and stop (no refit, no
+                        // requantization); a skipped item gets a NaN in its s_new block
 };
 
 struct QuantArgs {

@@ -84,6 +84,7 @@ def lib() -> C.CDLL:
         "sq_decode_step": [P, P, I32, P, P, P, P, P, P, P],
         "sq_window_flush": [P, P, I32, P],
         "sq_decode_chunk": [P, P, I32, I32, P, P, P, P, P, P, P],
+        "sq_decode_step_split": [P, P, I32, P, P, P, P, P, P, P, P, P],
         "sq_pool_status": [P, C.POINTER(I32)],
         "sq_debug_decode_step_fp32": [P, P, I32, P, P, P, P, P, P, P, P],
         "sq_allocate_bits": [I32, P, P, C.c_float, I32, P, P],
@@ -159,6 +160,13 @@ def sq_decode_step(pool: int, slot_idx: int, batch: int, q: int, k: int, v: int,
                    beta: int, out: int, stream: int) -> None:
     _chk(lib().sq_decode_step(pool, slot_idx, batch, q, k, v, alpha, beta, out, stream),
          "sq_decode_step")
+
+
+def sq_decode_step_split(pool: int, slot_idx: int, batch: int, q: int, k: int, v: int,
+                         alpha: int, beta: int, out: int, staging: int, stream: int,
+                         side_stream: int) -> None:
+    _chk(lib().sq_decode_step_split(pool, slot_idx, batch, q, k, v, alpha, beta, out, staging,
+                                    stream, side_stream), "sq_decode_step_split")
 
 
 def sq_decode_chunk(pool: int, slot_idx: int, batch: int, n_tokens: int, q: int, k: int, v: int,
@@ -251,6 +259,13 @@ class StatePool:
             sq_decode_step(*args, self._stream())
         else:
             sq_debug_decode_step_fp32(*args, s_new.data_ptr(), self._stream())
+
+    def decode_step_split(self, slot_idx, q, k, v, alpha, beta, out, staging, side_stream):
+        """The step with the refit and requantization on `side_stream` (a torch stream)."""
+        sq_decode_step_split(self.handle, slot_idx.data_ptr(), slot_idx.numel(), q.data_ptr(),
+                             k.data_ptr(), v.data_ptr(), alpha.data_ptr(), beta.data_ptr(),
+                             out.data_ptr(), staging.data_ptr(), self._stream(),
+                             side_stream.cuda_stream)
 
     def decode_chunk(self, slot_idx, q, k, v, alpha, beta, out):
         """q, k [B][H][T][d_k], v [B][H][T][d_v], alpha [B][H][T](or [..][d_k]), beta

@@ -60,6 +60,7 @@ class Workload:
     window: int = 1
     n_outliers: int = 0
     tokens: int = 1                # tokens per call (> 1: the multi-token chunk step)
+    side_stream: bool = False      # refit + requantize on a second stream (the split step)
     init_std: float = 0.1
     notes: str = field(default="", compare=False)
 
@@ -158,7 +159,7 @@ class Workload:
 
 
 # The workloads: a tiny oracle check, a GDN layer, a KDA layer, a serving pool, the windowed
-# variant and the GDN layer in 8-token chunks. Bit mixes: averages are over the non-pivot units.
+# variant, the GDN layer in 8-token chunks and the GDN layer with the side-stream split. Bit mixes: averages are over the non-pivot units.
 WORKLOADS = {
     "tiny": Workload(
         name="tiny", batch=2, n_heads=2, d_k=16, d_v=16, steps=8, gate=GATE_SCALAR,
@@ -190,6 +191,12 @@ WORKLOADS = {
         alpha_min=0.9, tokens=8,
         notes="the GDN layer advanced 8 tokens per call (prefill / speculative decode chunk), "
               "requantized once per call"),
+    "split": Workload(
+        name="split", batch=64, n_heads=32, d_k=128, d_v=128, steps=256, gate=GATE_SCALAR,
+        unit=UNIT_HEAD, io_dtype=IO_BF16, mix=((4, 10), (6, 10), (8, 10)), n_pivots=2, seed=1,
+        alpha_min=0.9, side_stream=True,
+        notes="the GDN layer with the update on one stream (fp32 state to a staging buffer) "
+              "and the refit + requantization on a second"),
 }
 
 

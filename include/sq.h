@@ -160,6 +160,22 @@ SQ_API sq_status sq_decode_step(sq_pool* pool, const int32_t* slot_idx, int32_t 
                          float* out, void* stream);
 
 /*
+ * The decode step split over two streams, for comparison with the fused sq_decode_step ([SQ-E]
+ * experimental-setup paragraph: the scale fit and compression run on a side stream). On
+ * `stream` one kernel unpacks, updates and writes out (as sq_decode_step) and writes the updated
+ * fp32 state to `staging`; on `side_stream`, after it, the fit and requantization of
+ * sq_quantize_fp32_state turn `staging` back into the slots. Every later call on this pool
+ * (any entry point, any stream) first waits for that requantization on the GPU.
+ *   staging (device, caller-owned scratch) fp32 [batch][n_heads][d_k][d_v], 16-byte aligned;
+ *   the caller must not touch it until the side stream's work has finished.
+ * Other arguments as sq_decode_step; window == 1 pools only (SQ_ERR_UNSUPPORTED otherwise).
+ * A request-head with a non-finite input keeps its bytes (SQ_FLAG_NONFINITE). */
+SQ_API sq_status sq_decode_step_split(sq_pool* pool, const int32_t* slot_idx, int32_t batch,
+                                      const void* q, const void* k, const void* v,
+                                      const float* alpha, const float* beta, float* out,
+                                      float* staging, void* stream, void* side_stream);
+
+/*
  * n_tokens consecutive tokens of each request in one call (prefill, or speculative decode into a
  * quantized state): the state is read from the pool once, advanced through the tokens in fp32 on
  * chip, and refit and requantized once, after the last token. Each token's update and output
