@@ -31,6 +31,14 @@ struct sq_pool {
   bool side_pending = false;
 };
 
+namespace sq {
+void pool_dims(const sq_pool* p, int* n_heads, int* d_k, int* d_v) {
+  *n_heads = p->L.n_heads;
+  *d_k = p->L.d_k;
+  *d_v = p->L.d_v;
+}
+}  // namespace sq
+
 namespace {
 
 bool width_ok(int b) { return b == 2 || b == 4 || b == 6 || b == 8 || b == 16; }

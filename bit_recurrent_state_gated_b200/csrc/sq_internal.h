@@ -3,6 +3,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+struct sq_pool;
+
 namespace sq {
 
 constexpr int kThreads = 256;  // 8 warps; warp w owns key rows [16w, 16w+16)
@@ -84,6 +86,8 @@ cudaError_t launch_window_step(const StepArgs& a, int gate, int io, int num_sms,
                                cudaStream_t st);
 cudaError_t launch_window_flush(const StepArgs& a, int num_sms, cudaStream_t st);
 cudaError_t launch_chunk(const StepArgs& a, int gate, int io, int num_sms, cudaStream_t st);
+// Heads and tile shape of a pool (for entry points outside the pool's own file).
+void pool_dims(const sq_pool* p, int* n_heads, int* d_k, int* d_v);
 constexpr int kMaxChunkTokens = 16;
 
 }  // namespace sq

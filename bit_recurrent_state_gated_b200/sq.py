@@ -85,6 +85,7 @@ def lib() -> C.CDLL:
         "sq_window_flush": [P, P, I32, P],
         "sq_decode_chunk": [P, P, I32, I32, P, P, P, P, P, P, P],
         "sq_decode_step_split": [P, P, I32, P, P, P, P, P, P, P, P, P],
+        "sq_decode_step_split_static": [P, P, I32, P, P, P, P, P, P, P],
         "sq_pool_status": [P, C.POINTER(I32)],
         "sq_debug_decode_step_fp32": [P, P, I32, P, P, P, P, P, P, P, P],
         "sq_allocate_bits": [I32, P, P, C.c_float, I32, P, P],
@@ -167,6 +168,14 @@ def sq_decode_step_split(pool: int, slot_idx: int, batch: int, q: int, k: int, v
                          side_stream: int) -> None:
     _chk(lib().sq_decode_step_split(pool, slot_idx, batch, q, k, v, alpha, beta, out, staging,
                                     stream, side_stream), "sq_decode_step_split")
+
+
+def sq_decode_step_split_static(pool: int, slot_idx: int, batch: int, q: int, k: int, v: int,
+                                alpha: int, beta: int, out: int, stream: int) -> None:
+    """The split step with libsq's own 32 MiB staging array (for callers that cannot
+    allocate device memory)."""
+    _chk(lib().sq_decode_step_split_static(pool, slot_idx, batch, q, k, v, alpha, beta, out,
+                                           stream), "sq_decode_step_split_static")
 
 
 def sq_decode_chunk(pool: int, slot_idx: int, batch: int, n_tokens: int, q: int, k: int, v: int,

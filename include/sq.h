@@ -176,6 +176,26 @@ SQ_API sq_status sq_decode_step_split(sq_pool* pool, const int32_t* slot_idx, in
                                       float* staging, void* stream, void* side_stream);
 
 /*
+ * sq_decode_step_split for callers that cannot allocate device memory (a serving engine that
+ * hands all device memory to its own allocator at start-up, a host whose memory plan is fixed
+ * before the first request): the staging state lives in a static device array that libsq
+ * owns, 32 MiB on every GPU that loads the library, held until the process exits. This entry
+ * point allocates nothing. The pages have no counterpart: it only serves such callers.
+ *   batch * n_heads * d_k * d_v * 4 bytes must fit in 32 MiB (512 request-heads at
+ *   d = 128); larger batches return SQ_ERR_INVALID_ARG.
+ * Both halves (update, then refit + requantize) run on `stream`. The first call on a device
+ * (with that device current) looks up the array's device address; make that first call
+ * before any stream capture. All calls in the process share the one array and it keeps the
+ * last call's contents (nothing in it needs to start at zero: each call writes every tile it
+ * reads back); calls that can run at the same time on the GPU (different streams, different
+ * pools) race on it and must be ordered by the caller. Other arguments and errors as
+ * sq_decode_step_split. */
+SQ_API sq_status sq_decode_step_split_static(sq_pool* pool, const int32_t* slot_idx,
+                                             int32_t batch, const void* q, const void* k,
+                                             const void* v, const float* alpha,
+                                             const float* beta, float* out, void* stream);
+
+/*
  * n_tokens consecutive tokens of each request in one call (prefill, or speculative decode into a
  * quantized state): the state is read from the pool once, advanced through the tokens in fp32 on
  * chip, and refit and requantized once, after the last token. Each token's update and output
