@@ -43,6 +43,8 @@ from bit_recurrent_state_gated_b200 import workloads as W  # noqa: E402
 METRIC = "quantized delta-rule decode: request-steps/s and state HBM GB/s vs peak"
 UNIT = "request-steps/s"
 L2_FLUSH_BYTES = 256 << 20  # > 126 MB of L2
+L2_BYTES = 126 << 20
+E2E_SETS = 8
 
 
 def parse():
@@ -270,18 +272,18 @@ def run_ours(args, info):
                               device="cuda")
         side = torch.cuda.Stream()
 
-    def call(q, k, v, a, b):
+    def call(q, k, v, a, b, si_ptr=None, out_ptr=None):
+        si_ptr = si.data_ptr() if si_ptr is None else si_ptr
+        out_ptr = out.data_ptr() if out_ptr is None else out_ptr
         if wl.side_stream:
-            sq.sq_decode_step_split(pool.handle, si.data_ptr(), wl.batch, q, k, v, a, b,
-                                    out.data_ptr(), staging.data_ptr(), st_handle,
-                                    side.cuda_stream)
+            sq.sq_decode_step_split(pool.handle, si_ptr, wl.batch, q, k, v, a, b, out_ptr,
+                                    staging.data_ptr(), st_handle, side.cuda_stream)
             stream.wait_stream(side)  # the step ends when the requantization has
         elif T > 1:
-            sq.sq_decode_chunk(pool.handle, si.data_ptr(), wl.batch, T, q, k, v, a, b,
-                               out.data_ptr(), st_handle)
+            sq.sq_decode_chunk(pool.handle, si_ptr, wl.batch, T, q, k, v, a, b, out_ptr,
+                               st_handle)
         else:
-            sq.sq_decode_step(pool.handle, si.data_ptr(), wl.batch, q, k, v, a, b,
-                              out.data_ptr(), st_handle)
+            sq.sq_decode_step(pool.handle, si_ptr, wl.batch, q, k, v, a, b, out_ptr, st_handle)
 
     def step(t):
         call(*(x.data_ptr() for x in sets_dev[t % n_sets]))
@@ -311,9 +313,12 @@ def run_ours(args, info):
     kernel_ms = [a.elapsed_time(b) for a, b in ev]
     dev_ms = dist.max_over_ranks(sum(kernel_ms), device="cuda")
 
-    # end to end: pinned host inputs -> device, step, o -> pinned host, every step. The step's
-    # q, k, v, alpha, beta sit back to back (256-byte aligned) in one pinned host buffer and
-    # cross in one copy into a device buffer of the same layout.
+    # end to end, through the same public calls: every step copies its q, k, v, alpha, beta from
+    # pinned host memory (back to back, 256-byte aligned, one copy) and reads its o back into
+    # pinned host memory. The copies run on their own streams, double-buffered, so step t+1's
+    # inputs cross while step t computes and step t's o crosses while step t+1 computes. L2:
+    # the steps rotate over E2E_SETS disjoint groups of slots (the batch's states, copied), so a
+    # group's state has left L2 before it is stepped again.
     offs, total = [], 0
     for a in sets_host[0]:
         offs.append(total)
@@ -324,28 +329,71 @@ def run_ours(args, info):
         for o, a in zip(offs, host):
             buf[o:o + a.numel() * a.element_size()].copy_(a.reshape(-1).view(torch.uint8))
         packed_host.append(buf)
-    d_packed = torch.empty(total, dtype=torch.uint8, device="cuda")
-    base = d_packed.data_ptr()
-    qp, kp, vp, ap, bp = (base + o for o in offs)
-    ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
+    state_set = wl.slots * pool.slot_bytes
+    n_rot = max(2, -(-2 * L2_BYTES // state_set))  # >= 2 L2s of state between reuses
+    n_rot = min(n_rot, E2E_SETS)
+    pool.close()
+    lay_r = sq.Layout(wl.slots * n_rot, wl.n_heads, wl.d_k, wl.d_v, wl.unit, wl.gate,
+                      wl.io_dtype, wl.fit_iters, wl.window, wl.n_outliers)
+    pool = sq.StatePool(lay_r, bits, wl.pivot_mask())
+    si_rot = []
+    for r in range(n_rot):
+        si_r = torch.from_numpy(si_np + r * wl.slots).cuda()
+        for c in range(0, wl.batch, 64):
+            S0 = torch.from_numpy(wl.initial_state(si_np[c:c + 64])).cuda()
+            pool.quantize(si_r[c:c + 64], S0)
+        si_rot.append(si_r)
+    d_in = [torch.empty(total, dtype=torch.uint8, device="cuda") for _ in range(2)]
+    outs = [torch.empty_like(out) for _ in range(2)]
+    outs_host = [torch.empty(out.shape, dtype=torch.float32).pin_memory() for _ in range(2)]
+    h2d_s, d2h_s = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in, ev_comp, ev_out = ([torch.cuda.Event() for _ in range(2)] for _ in range(3))
+
+    def issue_h2d(t):
+        i = t % 2
+        if t >= 2:
+            h2d_s.wait_event(ev_comp[i])  # step t-2 has finished reading d_in[i]
+        with torch.cuda.stream(h2d_s):
+            d_in[i].copy_(packed_host[(args.warmup + t) % n_sets], non_blocking=True)
+        ev_in[i].record(h2d_s)
+
+    def e2e_run(n):
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        h2d_s.wait_event(start)
+        issue_h2d(0)
+        for t in range(n):
+            i = t % 2
+            if t + 1 < n:
+                issue_h2d(t + 1)
+            stream.wait_event(ev_in[i])
+            if t >= 2:
+                stream.wait_event(ev_out[i])  # step t-2's o has left outs[i]
+            base = d_in[i].data_ptr()
+            call(*(base + o for o in offs), si_ptr=si_rot[t % n_rot].data_ptr(),
+                 out_ptr=outs[i].data_ptr())
+            ev_comp[i].record(stream)
+            d2h_s.wait_event(ev_comp[i])
+            with torch.cuda.stream(d2h_s):
+                outs_host[i].copy_(outs[i], non_blocking=True)
+            ev_out[i].record(d2h_s)
+        stream.wait_stream(h2d_s)
+        stream.wait_stream(d2h_s)
+        end.record(stream)
+        return start, end
+
+    e2e_run(args.warmup)
     dist.barrier()
     torch.cuda.synchronize()
-    for t in range(args.steps):
-        flush.zero_()
-        ev2[t][0].record(stream)
-        d_packed.copy_(packed_host[(args.warmup + t) % n_sets], non_blocking=True)
-        call(qp, kp, vp, ap, bp)
-        out_host.copy_(out, non_blocking=True)
-        ev2[t][1].record(stream)
+    start, end = e2e_run(args.steps)
     torch.cuda.synchronize()
     dist.barrier()
-    e2e_ms = dist.max_over_ranks(sum(a.elapsed_time(b) for a, b in ev2), device="cuda")
+    e2e_ms = dist.max_over_ranks(start.elapsed_time(end), device="cuda")
     st, flag = pool.status()
     if st != sq.SQ_OK:
         raise RuntimeError(f"device flag {flag} in the timed region")
     h2d = total
-    d2h = out_host.numel() * out_host.element_size()
+    d2h = outs_host[0].numel() * outs_host[0].element_size()
 
     total_req_steps = wl.batch * T * args.steps * info.world
     ab = algorithmic_bytes(wl, pool.slot_bytes)
@@ -388,7 +436,12 @@ def run_ours(args, info):
                      "kernel": kernel,
                      "mean_launch_us": mean_launch_s * 1e6},
         "e2e": {"value": total_req_steps / (e2e_ms / 1e3), "unit": UNIT,
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e2e_ms / args.steps,
+                "l2": f"steps rotate over {n_rot} disjoint slot groups "
+                      f"({n_rot * state_set / 2**20:.0f} MiB of state)",
+                "copies": "own streams, double-buffered (inputs of step t+1 and o of step t "
+                          "cross while step t / t+1 computes)"},
         "gpu_launches": args.steps * (2 if wl.side_stream else 1),
         "clocks": clocks.summary(),
     }
