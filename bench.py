@@ -401,7 +401,7 @@ def run_ours(args, info):
     achieved = ab["total"] * wl.batch * T / mean_launch_s / 1e9
     peak, peak_kind = peaks()
     kernel = ("k_chunk" if T > 1 else "k_window" if wl.window > 1 else
-              "k_decode (update only) + k_quantize" if wl.side_stream else "k_decode")
+              "k_decode_k_quantize" if wl.side_stream else "k_decode")
     traffic = profiled_traffic(args.workload, kernel)
     res = {
         "metric": METRIC,
