@@ -82,4 +82,10 @@ def test_calls_on_null_pool_rejected(lib):
         sq.sq_quantize_fp32_state(0, 16, 1, 16, 0)
     with pytest.raises(sq.SqError):
         sq.sq_pool_info(0, 1)
+    with pytest.raises(sq.SqError):
+        sq.sq_decode_chunk(0, 16, 1, 4, 16, 16, 16, 16, 16, 16, 0)
+    with pytest.raises(sq.SqError):
+        sq.sq_decode_step_split(0, 16, 1, 16, 16, 16, 16, 16, 16, 16, 0, 0)
+    with pytest.raises(sq.SqError):
+        sq.sq_decode_step_split_static(0, 16, 1, 16, 16, 16, 16, 16, 16, 0)
     sq.sq_state_pool_destroy(0)

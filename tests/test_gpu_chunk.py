@@ -96,6 +96,18 @@ def test_chunk_lockstep(name, T):
     assert mis <= max(1, 1e-4 * tot), f"{mis} of {tot} codes differ"
 
 
+@pytest.mark.parametrize("name", ["gdn-s", "kda-d64"])
+def test_chunk_rollout_256_tokens(name):
+    """32 chunks of 8 tokens, each checked against the oracle from the GPU's own bytes."""
+    case = G.GpuCase(CASES[name])
+    mis = tot = 0
+    for c in range(32):
+        m, n = chunk_lockstep(case, case.wl.chunk_inputs(8 * c, 8), what=f"chunk {c}")
+        mis, tot = mis + m, tot + n
+    assert mis <= max(1, 1e-4 * tot), f"{mis} of {tot} codes differ"
+    assert case.pool.status() == (sq.SQ_OK, 0)
+
+
 def test_one_token_chunk_is_the_decode_step():
     wl = CASES["gdn-s"]
     a, b = G.GpuCase(wl), G.GpuCase(wl)

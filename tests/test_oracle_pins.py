@@ -494,3 +494,41 @@ def test_window_flush_cadence(oracle):
     pool.window_flush(si)
     assert not np.array_equal(pool.data, prev)
     assert np.all(pool.count[si] == 0)
+
+
+@pytest.mark.parametrize("name", ["gdn", "kda"])
+def test_chunk_is_dense_recurrence_then_one_quantize(oracle, name):
+    """The chunk step's oracle (the windowed oracle with W = T, no compensation entries): after
+    T tokens its block is the quantization of the exact T-token recurrence from the
+    dequantized state, rounded once to fp32 (numpy dense form, fp64), and o at every token
+    is that recurrence's M_t^T q_t."""
+    T = 5
+    wl = W.small(name, batch=2, n_heads=2, d=16).scaled(window=T)
+    pool, si = _pool_case(oracle, wl)
+    M = pool.dequantize(si).astype(np.float64)
+    I = np.eye(wl.d_k)
+    for t in range(T):
+        x = wl.step_inputs(t)
+        o = pool.window_step(si, x["q"], x["k"], x["v"], x["alpha"], x["beta"])
+        for b in range(len(si)):
+            for h in range(wl.n_heads):
+                k = x["k"][b, h].astype(np.float64)
+                D = np.diag(x["alpha"][b, h]) if wl.gate == W.GATE_DIAG else x["alpha"][b, h] * I
+                M[b, h] = (I - x["beta"][b, h] * np.outer(k, k)) @ D @ M[b, h] \
+                    + x["beta"][b, h] * np.outer(k, x["v"][b, h])
+                np.testing.assert_allclose(o[b, h], M[b, h].T @ x["q"][b, h], rtol=1e-9,
+                                           atol=1e-11)
+    ref, _ = _pool_case(oracle, wl.scaled(window=1))
+    ref.quantize(si, M.astype(np.float32))
+    np.testing.assert_array_equal(pool.data.reshape(wl.slots, -1)[si],
+                                  ref.data.reshape(wl.slots, -1)[si])
+
+
+def test_chunk_inputs_stack_the_step_inputs():
+    wl = W.small("kda", batch=2, n_heads=3, d=16)
+    x = wl.chunk_inputs(4, 3)
+    for t in range(3):
+        s = wl.step_inputs(4 + t)
+        for name in s:
+            np.testing.assert_array_equal(x[name][:, :, t], s[name])
+    assert x["alpha"].shape == (2, 3, 3, 16) and x["beta"].shape == (2, 3, 3)
