@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
 #include <new>
 #include <vector>
 
@@ -26,6 +27,8 @@ struct sq_pool {
   int32_t* d_order = nullptr;
   int32_t* d_flag = nullptr;
   int device = 0, num_sms = 0;
+  float* d_rho = nullptr;  // row impact weights [H][d_k] (sq_pool_set_row_impact)
+  bool has_rho = false;
   // side-stream split: the last split's requantization, which later calls on the pool wait for
   cudaEvent_t ev_update = nullptr, ev_side = nullptr;
   bool side_pending = false;
@@ -184,6 +187,7 @@ sq::StepArgs step_args(sq_pool* p, const int32_t* slot_idx, int32_t batch, const
   a.side_head_bytes = (int64_t)p->side_head_bytes;
   a.window = p->L.window;
   a.n_outliers = p->L.n_outliers;
+  a.rho = p->has_rho ? p->d_rho : nullptr;
   return a;
 }
 
@@ -209,6 +213,7 @@ sq::QuantArgs quant_args(sq_pool* p, const int32_t* slot_idx, int32_t n, const f
   a.side = p->side_slot_bytes ? p->base + (size_t)p->L.n_slots * p->slot_bytes : nullptr;
   a.side_slot_bytes = (int64_t)p->side_slot_bytes;
   a.side_head_bytes = (int64_t)p->side_head_bytes;
+  a.rho = p->has_rho ? p->d_rho : nullptr;
   return a;
 }
 
@@ -305,6 +310,7 @@ sq_status sq_state_pool_destroy(sq_pool* pool) {
   cudaFree(pool->d_srows);
   cudaFree(pool->d_flag);
   cudaFree(pool->d_order);
+  cudaFree(pool->d_rho);
   if (pool->ev_update) cudaEventDestroy(pool->ev_update);
   if (pool->ev_side) cudaEventDestroy(pool->ev_side);
   delete pool;
@@ -421,6 +427,34 @@ sq_status sq_window_flush(sq_pool* pool, const int32_t* slot_idx, int32_t n, voi
   const sq::StepArgs a = step_args(pool, slot_idx, n, nullptr, nullptr, nullptr, nullptr,
                                    nullptr, nullptr, nullptr);
   return cuda_status(sq::launch_window_flush(a, pool->num_sms, static_cast<cudaStream_t>(stream)));
+}
+
+sq_status sq_pool_set_row_impact(sq_pool* pool, const float* impact) {
+  if (!pool) return SQ_ERR_INVALID_ARG;
+  if (!impact) {
+    pool->has_rho = false;
+    return SQ_OK;
+  }
+  const int H = pool->L.n_heads, dk = pool->L.d_k;
+  std::vector<float> rho((size_t)H * dk);
+  for (int h = 0; h < H; ++h) {
+    double mx = 0.0;
+    for (int i = 0; i < dk; ++i) {
+      const double x = impact[(size_t)h * dk + i];
+      if (!(x > 0.0) || !std::isfinite(x)) return SQ_ERR_INVALID_ARG;
+      mx = x > mx ? x : mx;
+    }
+    for (int i = 0; i < dk; ++i)
+      rho[(size_t)h * dk + i] = (float)((double)impact[(size_t)h * dk + i] / mx);
+  }
+  cudaError_t e = cudaDeviceSynchronize();  // no kernel of this pool may still read the table
+  if (e == cudaSuccess && !pool->d_rho)
+    e = cudaMalloc(&pool->d_rho, rho.size() * sizeof(float));
+  if (e == cudaSuccess)
+    e = cudaMemcpy(pool->d_rho, rho.data(), rho.size() * sizeof(float), cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return cuda_status(e);
+  pool->has_rho = true;
+  return SQ_OK;
 }
 
 sq_status sq_pool_status(sq_pool* pool, int32_t* device_flag) {

@@ -381,8 +381,10 @@ __device__ __forceinline__ void pass_b(const Ctx<FULL>& c, const float4& cv, con
 // Row scales from the row maxima in S_RT, one row per lane: m = t max |tile row|,
 // r = max(m / Q, 2^-14) (at most the largest fp16), w = 1 / (r Q); S_W gets t w, the factor of
 // the tile row in the column passes; fp16 rows get r = w = 0. Returns the lane's r.
+// rho: this row's impact weight in (0, 1] (1 without an impact table): the scale widens to
+// min(fl(q / rho), 65504) when that exceeds q = m / Q.
 template <bool FULL>
-__device__ __forceinline__ float row_scales(const Ctx<FULL>& c, bool check) {
+__device__ __forceinline__ float row_scales(const Ctx<FULL>& c, bool check, float rho) {
   const int p = c.row0() + c.lane;
   float r = 0.f, w = 0.f;
   if (p < c.dk()) {
@@ -393,7 +395,9 @@ __device__ __forceinline__ float row_scales(const Ctx<FULL>& c, bool check) {
       const float t = sp<float>(S_TR)[p];
       const float rq = div_q(__fmul_rn(t, sp<float>(S_RT)[p]), Q, inv_q);  // exactly m / Q
       if (check && !(rq < 65520.f)) atomicOr(&c.flags[F_RANGE], 1);
-      r = fminf(fmaxf(rq, kScaleFloor), 65504.f);
+      r = fmaxf(rq, kScaleFloor);
+      if (rho != 1.f) r = fmaxf(r, fminf(__fdiv_rn(rq, rho), 65504.f));
+      r = fminf(r, 65504.f);
       w = __fmul_rn(t, rcp_approx(__fmul_rn(r, Q)));
     }
   }
@@ -782,6 +786,7 @@ __global__ void __launch_bounds__(kT, kMaxCtasPerSm) k_decode(const StepArgs a) 
     // columns' old scale and v, before the stage is handed back ----
     float4 cv = make_float4(1.f, 1.f, 1.f, 1.f), vv = make_float4(0.f, 0.f, 0.f, 0.f);
     float4 icv = make_float4(1.f, 1.f, 1.f, 1.f);
+    float rho = 1.f;  // this row's impact weight (used by the refit, loaded early)
     if (hdr.valid) {
       bool bad_in = false, bad_a = false;
       float kqp = 0.f;
@@ -797,6 +802,7 @@ __global__ void __launch_bounds__(kT, kMaxCtasPerSm) k_decode(const StepArgs a) 
         }
         sp<uint32_t>(S_RD)[p] = d;
         const int i = rd_row(d);
+        if (a.rho) rho = __ldg(a.rho + (size_t)hdr.h * dk + i);
         const float ki = ld_io(st + P.k_off, IO, i), qi = ld_io(st + P.q_off, IO, i);
         const float ai = GATE == 0 ? hdr.alpha : reinterpret_cast<const float*>(st + P.al_off)[i];
         bad_in |= !isfinite(ki) || !isfinite(qi) || !isfinite(ai);
@@ -915,13 +921,13 @@ __global__ void __launch_bounds__(kT, kMaxCtasPerSm) k_decode(const StepArgs a) 
       __syncthreads();
       continue;
     }
-    float r = row_scales(c, true);
+    float r = row_scales(c, true, rho);
     col_pass(c, sp<float>(S_REDC));
     __syncthreads();  // barrier 2
     float4 cm = max4(sp<float>(S_REDC), c.lane);
     for (int f = 1; f < a.fit_iters; ++f) {
       row_pass(c, make_float4(rcp_approx(cm.x), rcp_approx(cm.y), rcp_approx(cm.z), rcp_approx(cm.w)));
-      r = row_scales(c, false);
+      r = row_scales(c, false, rho);
       float* red = sp<float>(S_REDC) + (f & 1) * kW * kMaxD;
       col_pass(c, red);
       __syncthreads();  // barrier 3 (fit_iters = 2)
@@ -1131,7 +1137,7 @@ template <int GATE, bool FULL, bool ROWS>
 __device__ __forceinline__ void window_fold(const Ctx<FULL>& c, const StepArgs& a, const uint8_t* blk,
                                             const float* terms, int cnt, int mode,
                                             const float4& cv, const float4& bv, uint8_t* dst,
-                                            int32_t* count) {
+                                            float rho, int32_t* count) {
   const int dk = c.dk(), dv = c.dv(), tid = c.tid, lane = c.lane;
   const bool pivot_head = !ROWS && mode == MODE_PIVOT;
   const int n_out = pivot_head ? 0 : a.n_outliers;
@@ -1404,13 +1410,13 @@ __device__ __forceinline__ void window_fold(const Ctx<FULL>& c, const StepArgs& 
     if (of) atomicOr(&c.flags[F_RANGE], 1);
     __syncwarp();
   }
-  float r = row_scales(c, true);
+  float r = row_scales(c, true, rho);
   col_pass(c, sp<float>(S_REDC));
   __syncthreads();
   float4 cm = max4(sp<float>(S_REDC), lane);
   for (int f = 1; f < a.fit_iters; ++f) {
     row_pass(c, make_float4(rcp_approx(cm.x), rcp_approx(cm.y), rcp_approx(cm.z), rcp_approx(cm.w)));
-    r = row_scales(c, false);
+    r = row_scales(c, false, rho);
     float* red = sp<float>(S_REDC) + (f & 1) * kW * kMaxD;
     col_pass(c, red);
     __syncthreads();
@@ -1593,7 +1599,7 @@ __global__ void __launch_bounds__(kT, 3) k_window(const StepArgs a) {
     const bool pivot_head = !ROWS && mode == MODE_PIVOT;
 
     // ---- setup: thread t takes processing row t and value column t ----
-    float tc = 1.f, tv = 0.f;
+    float tc = 1.f, tv = 0.f, rho = 1.f;
     float4 cv = make_float4(1.f, 1.f, 1.f, 1.f);
     if (hdr.valid) {
       bool bad_in = false, under = false;
@@ -1610,6 +1616,7 @@ __global__ void __launch_bounds__(kT, 3) k_window(const StepArgs a) {
         }
         sp<uint32_t>(S_RD)[p] = d;
         const int i = rd_row(d);
+        if (a.rho) rho = __ldg(a.rho + (size_t)hdr.h * dk + i);
         sp<int>(W_INV)[i] = p;
         const float ki = ld_io(st + P.k_off, IO, i), qi = ld_io(st + P.q_off, IO, i);
         const float ai = GATE == 0 ? hdr.alpha : reinterpret_cast<const float*>(st + P.al_off)[i];
@@ -1769,7 +1776,7 @@ __global__ void __launch_bounds__(kT, 3) k_window(const StepArgs a) {
         float4 bv = make_float4(0.f, 0.f, 0.f, 0.f);
         if (c.act()) bv = *reinterpret_cast<const float4*>(sp<float>(W_OU) + 4 * c.lane);
         uint8_t* dst = a.pool + (size_t)hdr.slot * a.slot_bytes + hdr.off;
-        window_fold<GATE, FULL, ROWS>(c, a, blk, terms, cnt, mode, cv, bv, dst,
+        window_fold<GATE, FULL, ROWS>(c, a, blk, terms, cnt, mode, cv, bv, dst, rho,
                                       reinterpret_cast<int32_t*>(side));
       }
     }
@@ -2094,7 +2101,7 @@ __global__ void __launch_bounds__(kT, ROWS ? 4 : 3) k_chunk(const StepArgs a) {
     const float* as = reinterpret_cast<const float*>(st + P.as_off);
 
     // ---- token-independent setup, and every token's inputs checked ----
-    float tc = 1.f, g = 1.f, A = 1.f;
+    float tc = 1.f, g = 1.f, A = 1.f, rho = 1.f;
     float4 cv = make_float4(1.f, 1.f, 1.f, 1.f), icv = make_float4(1.f, 1.f, 1.f, 1.f);
     int i = 0;
     if (hdr.valid) {
@@ -2111,6 +2118,7 @@ __global__ void __launch_bounds__(kT, ROWS ? 4 : 3) k_chunk(const StepArgs a) {
         }
         sp<uint32_t>(S_RD)[p] = d;
         i = rd_row(d);
+        if (a.rho) rho = __ldg(a.rho + (size_t)hdr.h * dk + i);
         sp<int>(W_INV)[i] = p;
         sp<float>(S_TR)[p] = 1.f;  // the fold's tile holds the state itself
         A = (!pivot_head && rd_width(d) != 16) ? __half2float(reinterpret_cast<const __half*>(blk)[i]) : 1.f;
@@ -2258,7 +2266,8 @@ __global__ void __launch_bounds__(kT, ROWS ? 4 : 3) k_chunk(const StepArgs a) {
       float4 bv = make_float4(0.f, 0.f, 0.f, 0.f);
       if (c.act()) bv = *reinterpret_cast<const float4*>(sp<float>(W_OU) + 4 * c.lane);
       uint8_t* dst = a.pool + (size_t)hdr.slot * a.slot_bytes + hdr.off;
-      window_fold<GATE, FULL, ROWS>(c, a, blk, terms, T - 1 - t0, mode, cv, bv, dst, &dummy_count);
+      window_fold<GATE, FULL, ROWS>(c, a, blk, terms, T - 1 - t0, mode, cv, bv, dst, rho,
+                                    &dummy_count);
     }
     __syncthreads();
   }

@@ -56,6 +56,7 @@ struct StepArgs {
   int64_t side_slot_bytes, side_head_bytes;
   int32_t window, n_outliers;
   int32_t n_tok;  // tokens of a chunk (sq_decode_chunk)
+  const float* rho;  // null, or [H][d_k] row impact / the head's largest (sq_pool_set_row_impact)
   int32_t update_only;  // with s_new: write the updated fp32 state and stop (no refit, no
                         // requantization); a skipped item gets a NaN in its s_new block
 };
@@ -67,6 +68,7 @@ struct QuantArgs {
   const int32_t* slot_idx;
   int32_t n;
   const float* S;  // quantize: input; dequantize: output (cast away const)
+  const float* rho;  // null, or [H][d_k] row impact weights (as StepArgs::rho)
   float* S_out;
   const HeadDesc* heads;
   const uint32_t* rows;

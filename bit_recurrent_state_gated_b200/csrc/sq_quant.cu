@@ -50,7 +50,9 @@ __global__ void __launch_bounds__(kThreads) k_quantize(const QuantArgs a) {
     return;
   }
   uint8_t* dst = a.pool + (size_t)slot * a.slot_bytes + hd.off;
-  const bool ok = quantize_tile(S, dst, hd, rows, a.n_outliers, a.fit_iters, warp, lane, dk, dv, sm);
+  const float* rho = a.rho ? a.rho + (size_t)h * dk : nullptr;
+  const bool ok = quantize_tile(S, dst, hd, rows, rho, a.n_outliers, a.fit_iters, warp, lane, dk,
+                                dv, sm);
   if (!ok && tid == 0) atomicOr(a.flag, SQ_FLAG_RANGE_BIT);
   if (a.side && tid == 0)  // close this head's window
     *reinterpret_cast<int32_t*>(a.side + (size_t)slot * a.side_slot_bytes +

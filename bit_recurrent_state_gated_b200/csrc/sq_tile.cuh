@@ -43,10 +43,13 @@ __device__ __forceinline__ int q_of_width(int b) { return b == 16 ? 0 : (1 << (b
 // w_i = fl(1 / fl(r_i Q_i)); c_j = max(max_i fl(|S_ij| w_i), 2^-14). Rows with Q = 0 (fp16
 // pivot rows) get w = 0 and drop out of the column maxima; zeroed elements (outliers, idle
 // lanes) contribute nothing. On return rowR[i] = r_i and col[COL_X][j] = c_j.
+// Row impact (rho, per row of the head, in (0, 1], or null): a row's scale widens to
+// min(fl(q_i / rho_i), 65504) when that is larger than q_i = fl(m_i / Q_i), so its w_i shrinks
+// and the column scales follow the high-impact rows.
 __device__ __forceinline__ void fit_scales(const float (&S)[kRows][4], int fit_iters, int warp,
                                            int lane, int dk, int dv, const uint32_t* rows,
-                                           float* rowW, float* rowR, float* rowtmp, float* red,
-                                           float* col) {
+                                           const float* rho, float* rowW, float* rowR,
+                                           float* rowtmp, float* red, float* col) {
   float inv_c[4] = {1.f, 1.f, 1.f, 1.f};
   float* tmp = rowtmp + warp * kRows;
   for (int it = 0; it < fit_iters; ++it) {
@@ -73,7 +76,9 @@ __device__ __forceinline__ void fit_scales(const float (&S)[kRows][4], int fit_i
         const int Q = q_of_width(row_width(rows[i]));
         float r = 0.f, w = 0.f;
         if (Q > 0) {
-          r = fmaxf(__fdiv_rn(tmp[lane], (float)Q), kScaleFloor);
+          const float q = __fdiv_rn(tmp[lane], (float)Q);
+          r = fmaxf(q, kScaleFloor);
+          if (rho) r = fmaxf(r, fminf(__fdiv_rn(q, rho[i]), 65504.f));
           w = __frcp_rn(__fmul_rn(r, (float)Q));
         }
         rowR[i] = r;
@@ -479,8 +484,8 @@ __device__ __forceinline__ void select_top_fast(const float (&S)[kRows][4], int 
 // stored) on an fp16 range overflow. Contains __syncthreads; sm.misc[0] must be 0 on entry.
 __device__ __forceinline__ bool quantize_tile(float (&S)[kRows][4], uint8_t* dst,
                                               const HeadDesc& hd, const uint32_t* rows,
-                                              int n_out, int fit_iters, int warp, int lane,
-                                              int dk, int dv, TileSmem& sm) {
+                                              const float* rho, int n_out, int fit_iters,
+                                              int warp, int lane, int dk, int dv, TileSmem& sm) {
   if (hd.pivot_head) return store_pivot_head(S, dst, warp, lane, dk, dv, &sm.misc[0]);
   if (n_out > 0) {
     uint64_t sel = 0;
@@ -493,7 +498,8 @@ __device__ __forceinline__ bool quantize_tile(float (&S)[kRows][4], uint8_t* dst
     if ((int)threadIdx.x < n_out && __hisinf(__float2half_rn(sm.oval[threadIdx.x])))
       atomicOr(&sm.misc[0], 1);
   }
-  fit_scales(S, fit_iters, warp, lane, dk, dv, rows, sm.rowW, sm.rowR, sm.rowtmp, sm.red, sm.col);
+  fit_scales(S, fit_iters, warp, lane, dk, dv, rows, rho, sm.rowW, sm.rowR, sm.rowtmp, sm.red,
+             sm.col);
   const bool ok = requant_store_any(mode_of(hd), S, dst, rows, warp, lane, dk, dv, sm.rowR,
                                     sm.rowIR, sm.col, &sm.misc[0]);
   if (ok && n_out > 0 && (int)threadIdx.x < n_out) {

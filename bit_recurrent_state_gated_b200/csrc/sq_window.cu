@@ -94,7 +94,8 @@ __device__ __forceinline__ void flush_tile(const StepArgs& a, TileSmem& ts, cons
                                            const float* terms, int nterms, const float* g,
                                            bool add_new, const float* kk, const float* bcol,
                                            uint8_t* dst, const HeadDesc& hd,
-                                           const uint32_t* rows, int32_t* count) {
+                                           const uint32_t* rows, const float* rho,
+                                           int32_t* count) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, dk = a.dk, dv = a.dv;
   float S[kRows][4];
   frozen_tile<true>(S, blk, hd, rows, a.n_outliers, warp, lane, dk, dv);
@@ -129,7 +130,8 @@ __device__ __forceinline__ void flush_tile(const StepArgs& a, TileSmem& ts, cons
   }
   if (tid == 0) ts.misc[0] = 0;
   __syncthreads();
-  const bool ok = quantize_tile(S, dst, hd, rows, a.n_outliers, a.fit_iters, warp, lane, dk, dv, ts);
+  const bool ok = quantize_tile(S, dst, hd, rows, rho, a.n_outliers, a.fit_iters, warp, lane, dk,
+                                dv, ts);
   if (!ok && tid == 0) atomicOr(a.flag, SQ_FLAG_RANGE_BIT);
   if (tid == 0) *count = 0;
 }
@@ -158,7 +160,8 @@ __global__ void __launch_bounds__(kThreads) k_window_flush(const StepArgs a) {
   copy16(terms, side + 16 + 4 * dk, (uint32_t)cnt * (dk + dv) * 4, a.flag);
   copy16(sm.g, side + 16, dk * 4, a.flag);
   __syncthreads();
-  flush_tile(a, sm.t, blk, terms, cnt, sm.g, false, nullptr, nullptr, dst, hd, rows, count);
+  flush_tile(a, sm.t, blk, terms, cnt, sm.g, false, nullptr, nullptr, dst, hd, rows,
+             a.rho ? a.rho + (size_t)h * dk : nullptr, count);
   (void)tid;
 }
 

@@ -86,6 +86,7 @@ def lib() -> C.CDLL:
         "sq_decode_chunk": [P, P, I32, I32, P, P, P, P, P, P, P],
         "sq_decode_step_split": [P, P, I32, P, P, P, P, P, P, P, P, P],
         "sq_decode_step_split_static": [P, P, I32, P, P, P, P, P, P, P],
+        "sq_pool_set_row_impact": [P, P],
         "sq_pool_status": [P, C.POINTER(I32)],
         "sq_debug_decode_step_fp32": [P, P, I32, P, P, P, P, P, P, P, P],
         "sq_allocate_bits": [I32, P, P, C.c_float, I32, P, P],
@@ -176,6 +177,15 @@ def sq_decode_step_split_static(pool: int, slot_idx: int, batch: int, q: int, k:
     allocate device memory)."""
     _chk(lib().sq_decode_step_split_static(pool, slot_idx, batch, q, k, v, alpha, beta, out,
                                            stream), "sq_decode_step_split_static")
+
+
+def sq_pool_set_row_impact(pool: int, impact) -> None:
+    """impact: [n_heads][d_k] positive scores (host), or None to remove the weighting."""
+    if impact is None:
+        _chk(lib().sq_pool_set_row_impact(pool, None), "sq_pool_set_row_impact")
+        return
+    a = np.ascontiguousarray(np.asarray(impact, dtype=np.float32))
+    _chk(lib().sq_pool_set_row_impact(pool, a.ctypes.data), "sq_pool_set_row_impact")
 
 
 def sq_decode_chunk(pool: int, slot_idx: int, batch: int, n_tokens: int, q: int, k: int, v: int,
@@ -282,6 +292,9 @@ class StatePool:
         sq_decode_chunk(self.handle, slot_idx.data_ptr(), slot_idx.numel(), q.shape[2],
                         q.data_ptr(), k.data_ptr(), v.data_ptr(), alpha.data_ptr(),
                         beta.data_ptr(), out.data_ptr(), self._stream())
+
+    def set_row_impact(self, impact):
+        sq_pool_set_row_impact(self.handle, impact)
 
     def window_flush(self, slot_idx):
         sq_window_flush(self.handle, slot_idx.data_ptr(), slot_idx.numel(), self._stream())

@@ -218,6 +218,21 @@ SQ_API sq_status sq_decode_chunk(sq_pool* pool, const int32_t* slot_idx, int32_t
  * the window (no-op for a closed window). slot_idx (device) [n]. */
 SQ_API sq_status sq_window_flush(sq_pool* pool, const int32_t* slot_idx, int32_t n, void* stream);
 
+/*
+ * Row-impact weighting of the dual-axis fit ([SQ-E] experimental-setup paragraph: the row scale
+ * weighs the row's current size together with its impact score, and the column scale
+ * penalizes reconstruction error more in high-impact rows; the impact scores are fixed
+ * offline, [SQ-E] row-impact score paragraph). impact (host) fp32 [n_heads][d_k], every entry
+ * > 0 and finite, or NULL to remove the weighting. Reading taken (the pages print no
+ * formula): rho_i = impact_i / (largest impact of the head) in fp64, rounded to fp32; in
+ * every refit of the pool (decode step, chunk, window end, quantize, flush) the row scale
+ * becomes r_i = max(q_i, min(q_i / rho_i, 65504), 2^-14) with q_i = m_i / Q_i (m_i the row's
+ * max-abs over the current column scales), so low-impact rows take wider steps and the column
+ * scales follow the high-impact rows; no code leaves [-Q, Q]. Synchronizes the device;
+ * allocates a small device table on first use. SQ_ERR_INVALID_ARG for a bad entry (the
+ * previous weighting stays). */
+SQ_API sq_status sq_pool_set_row_impact(sq_pool* pool, const float* impact);
+
 /* Synchronize the device, read and clear the status word (*device_flag, may be NULL).
  * Returns SQ_OK, SQ_ERR_DEVICE_FLAG or SQ_ERR_TIMEOUT. */
 SQ_API sq_status sq_pool_status(sq_pool* pool, int32_t* device_flag);

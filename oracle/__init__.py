@@ -8,7 +8,7 @@ from __future__ import annotations
 
 import ctypes as C
 import os
-from dataclasses import dataclass
+from dataclasses import dataclass, field
 
 import numpy as np
 
@@ -25,7 +25,8 @@ class OracleError(RuntimeError):
 
 class _Layout(C.Structure):
     _fields_ = [(n, C.c_int32) for n in
-                ("n_heads", "d_k", "d_v", "unit", "gate", "fit_iters", "window", "n_outliers")]
+                ("n_heads", "d_k", "d_v", "unit", "gate", "fit_iters", "window", "n_outliers")
+                ] + [("rho", C.c_void_p)]
 
 
 @dataclass(frozen=True)
@@ -38,10 +39,24 @@ class Layout:
     fit_iters: int = 2
     window: int = 1
     n_outliers: int = 0
+    row_impact: object = field(default=None, compare=False, hash=False)  # [n_heads][d_k] > 0
+
+    def rho(self):
+        """Impact scores divided by the largest of their head (fp64 division, then fp32)."""
+        if self.row_impact is None:
+            return None
+        imp = np.asarray(self.row_impact, dtype=np.float64).reshape(self.n_heads, self.d_k)
+        assert np.all(np.isfinite(imp)) and np.all(imp > 0)
+        return np.ascontiguousarray((imp / imp.max(axis=1, keepdims=True)).astype(np.float32))
 
     def c(self) -> _Layout:
-        return _Layout(self.n_heads, self.d_k, self.d_v, self.unit, self.gate, self.fit_iters,
-                       self.window, self.n_outliers)
+        lay = _Layout(self.n_heads, self.d_k, self.d_v, self.unit, self.gate, self.fit_iters,
+                      self.window, self.n_outliers, None)
+        rho = self.rho()
+        if rho is not None:
+            lay.rho = rho.ctypes.data
+            lay.keep = rho  # the table lives as long as the structure
+        return lay
 
     @property
     def alpha_width(self) -> int:
@@ -66,7 +81,7 @@ def lib():
             "orc_unpack_row": [C.c_int, C.c_int, P, P],
             "orc_f32_to_f16_bits": [C.c_float],
             "orc_f16_bits_to_f32": [C.c_uint16],
-            "orc_fit": [C.c_int, C.c_int, C.c_int, P, P, P, P, P],
+            "orc_fit": [C.c_int, C.c_int, C.c_int, P, P, P, P, P, P],
             "orc_select_outliers": [C.c_int, C.c_int, P, P, C.c_int, P],
             "orc_quantize_head": [P, P, C.c_int, P, P],
             "orc_dequantize_head": [P, P, C.c_int, P, P],
@@ -148,15 +163,17 @@ def f32_to_f16_bits(x: float) -> int:
     return int(lib().orc_f32_to_f16_bits(float(x)))
 
 
-def fit(S: np.ndarray, qmax, fit_iters: int = 2, excluded=None):
+def fit(S: np.ndarray, qmax, fit_iters: int = 2, excluded=None, rho=None):
+    """(r, c) of the dual-axis fit; rho: optional per-row weights in (0, 1] (impact)."""
     S = np.ascontiguousarray(S, dtype=np.float32)
     dk, dv = S.shape
     q = np.ascontiguousarray(np.asarray(qmax, dtype=np.int32))
     ex = None if excluded is None else np.ascontiguousarray(np.asarray(excluded, dtype=np.uint8))
+    rh = None if rho is None else np.ascontiguousarray(np.asarray(rho, dtype=np.float32))
     r = np.zeros(dk, dtype=np.float32)
     c = np.zeros(dv, dtype=np.float32)
-    _chk(lib().orc_fit(dk, dv, fit_iters, _p(S), _p(q), None if ex is None else _p(ex), _p(r),
-                       _p(c)), "fit")
+    _chk(lib().orc_fit(dk, dv, fit_iters, _p(S), _p(q), None if ex is None else _p(ex),
+                       None if rh is None else _p(rh), _p(r), _p(c)), "fit")
     return r, c
 
 

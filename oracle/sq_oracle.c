@@ -26,7 +26,10 @@
  * Parity pins (tests/test_oracle_pins.py) cover every exported function: closed forms of the
  * delta rule, Proposition 1, quantize/dequantize idempotence, the half-step error bound, the
  * textbook special cases, brute force on 4x4 tiles, and a format-size check against the
- * compression ratios [SQ-E] prints. No function here is "parity unpinned".
+ * compression ratios [SQ-E] prints. One part is "parity unpinned": the row-impact weighting
+ * of orc_fit (rho != NULL), whose formula the pages do not print; the reading taken is pinned
+ * only by its special cases (a hand-worked 2 x 2 example, rho = 1 giving the plain fit, codes
+ * within [-Q, Q] and the half-step bound, monotone first alternation).
  */
 #include "sq_oracle.h"
 
@@ -165,9 +168,20 @@ void orc_unpack_row(int b, int n, const uint8_t* in, int32_t* u) {
  *     w_i = fl(1 / fl(r_i * Q_i));  c_j = max( max_i fl(|S_ij| * w_i) , 2^-14 )
  * Rows with qmax[i] == 0 (fp16 pivot rows) and elements with excluded[] set (outliers) take
  * no part. The caller rounds r and c to fp16 once, at the end.
+ *
+ * Impact weighting (rho != NULL; parity unpinned beyond its special cases, the pages print no
+ * formula). [SQ-E] experimental-setup paragraph: the row scale weighs the row's current size
+ * together with its impact score, and the column scale penalizes reconstruction error more in
+ * high-impact rows (wide range for large rows, finer resolution for important rows). Reading
+ * taken: with rho_i in (0, 1] the row's impact divided by the largest of its head,
+ *     r_i = max( fl(q_i / rho_i) capped at 65504 , q_i , 2^-14 ),  q_i = fl(m_i / Q_i),
+ * so a low-impact row takes a wider step than its own range needs, its w_i shrinks, and the
+ * column maxima c_j are set by the high-impact rows. No element leaves [-Q, Q] (every
+ * |S_ij| w_i <= c_j still holds), rho = 1 is the plain fit above, and scaling every rho_i of a
+ * head by one factor leaves r_i c_j unchanged up to rounding.
  * ---------------------------------------------------------------------------------------- */
 int orc_fit(int d_k, int d_v, int fit_iters, const float* S, const int32_t* qmax,
-            const uint8_t* excluded, float* r, float* c) {
+            const uint8_t* excluded, const float* rho, float* r, float* c) {
   float* inv_c = (float*)malloc(sizeof(float) * (size_t)d_v);
   float* w = (float*)malloc(sizeof(float) * (size_t)d_k);
   if (!inv_c || !w) {
@@ -192,7 +206,13 @@ int orc_fit(int d_k, int d_v, int fit_iters, const float* S, const int32_t* qmax
         if (a > m) m = a;
       }
       float ri = m / (float)qmax[i];
-      r[i] = ri > ORC_SCALE_FLOOR ? ri : ORC_SCALE_FLOOR;
+      float rr = ri > ORC_SCALE_FLOOR ? ri : ORC_SCALE_FLOOR;
+      if (rho) {
+        float wide = ri / rho[i];
+        if (wide > 65504.0f) wide = 65504.0f;
+        if (wide > rr) rr = wide;
+      }
+      r[i] = rr;
     }
     for (int i = 0; i < d_k; ++i) w[i] = qmax[i] ? 1.0f / (r[i] * (float)qmax[i]) : 0.0f;
     for (int j = 0; j < d_v; ++j) { /* column pass */
@@ -303,7 +323,7 @@ int orc_quantize_head(const orc_layout* L, const uint8_t* bits, int h, const flo
     if (st) goto done;
     for (int t = 0; t < L->n_outliers; ++t) excl[oidx[t]] = 1;
   }
-  orc_fit(dk, dv, L->fit_iters, S, qmax, excl, r, c);
+  orc_fit(dk, dv, L->fit_iters, S, qmax, excl, L->rho ? L->rho + (size_t)h * dk : NULL, r, c);
 
   uint8_t* r16p = block;
   uint8_t* c16p = block + 2 * (size_t)dk;

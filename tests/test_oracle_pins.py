@@ -532,3 +532,88 @@ def test_chunk_inputs_stack_the_step_inputs():
         for name in s:
             np.testing.assert_array_equal(x[name][:, :, t], s[name])
     assert x["alpha"].shape == (2, 3, 3, 16) and x["beta"].shape == (2, 3, 3)
+
+
+# ---- row-impact weighting of the fit (parity unpinned beyond these special cases) ----------
+
+def test_impact_worked_example(oracle):
+    """A 2 x 2 4-bit head worked by hand. S = [[4, 1], [1, 4]], impacts [4, 1] (rho = [1, 1/4]),
+    one alternation. Plain fit: r = [4/7, 4/7], c = [1, 1], codes [[7, 2], [2, 7]]. Weighted:
+    r_1 = 4 fl(4/7) (the low-impact row widens), w = [1/4, 1/16], so c_1 = max(1/4, 4/16) = 1/4:
+    row 0 becomes exact (codes [7, 7]) and row 1 takes the error (codes [0, 7])."""
+    S = np.array([[4.0, 1.0], [1.0, 4.0]], dtype=np.float32)
+    q7 = np.float32(4.0) / np.float32(7.0)
+    r, c = oracle.fit(S, [7, 7], fit_iters=1)
+    np.testing.assert_array_equal(r, [q7, q7])
+    np.testing.assert_array_equal(c, [1.0, 1.0])
+    r, c = oracle.fit(S, [7, 7], fit_iters=1, rho=[1.0, 0.25])
+    np.testing.assert_array_equal(r, [q7, 4 * q7])
+    np.testing.assert_array_equal(c, [1.0, 0.25])
+    for impact, want in ((None, [[7, 2], [2, 7]]), ([[4.0, 1.0]], [[7, 7], [0, 7]])):
+        lay = oracle.Layout(1, 2, 2, row_impact=impact, fit_iters=1)
+        blk = oracle.quantize_head(lay, [4], 0, S)
+        rb = oracle.row_bytes(4, 2)  # rows follow r16[2] | c16[2]
+        codes = [oracle.unpack_row(4, 2, blk[8 + rb * i:8 + rb * (i + 1)]) - 8 for i in range(2)]
+        np.testing.assert_array_equal(codes, want)
+
+
+def test_impact_of_ones_is_the_plain_fit(oracle):
+    """Equal impacts (rho = 1 everywhere) leave every byte as the unweighted fit makes it."""
+    wl = W.small("kda", batch=2, n_heads=2, d=32)
+    S = wl.initial_state(wl.slot_idx()) * 7.0
+    lay = G_layout(oracle, wl)
+    lay1 = G_layout(oracle, wl, row_impact=np.full((wl.n_heads, wl.d_k), 3.5))
+    for h in range(wl.n_heads):
+        np.testing.assert_array_equal(oracle.quantize_head(lay, wl.bits(), h, S[0, h]),
+                                      oracle.quantize_head(lay1, wl.bits(), h, S[0, h]))
+
+
+def G_layout(oracle, wl, **kw):
+    return oracle.Layout(wl.n_heads, wl.d_k, wl.d_v, wl.unit, wl.gate, wl.fit_iters, wl.window,
+                         wl.n_outliers, **kw)
+
+
+@pytest.mark.parametrize("name", ["gdn", "kda", "window"])
+def test_impact_codes_stay_in_range_and_error_bounded(oracle, name):
+    """Random impacts: every code within [-Q, Q] (no clipping) and every element of a
+    quantized row within half a step r16_i c16_j of its value (fp16 rounding of the scales
+    aside), as for the plain fit."""
+    wl = W.small(name, batch=1, n_heads=3, d=32)
+    rng = np.random.default_rng(11)
+    imp = rng.uniform(0.01, 1.0, (wl.n_heads, wl.d_k))
+    lay = G_layout(oracle, wl, row_impact=imp)
+    S = wl.initial_state(wl.slot_idx())[0] * 5.0
+    bits = wl.bits()
+    for h in range(wl.n_heads):
+        blk = oracle.quantize_head(lay, bits, h, S[h])
+        D = oracle.dequantize_head(lay, bits, h, blk)
+        widths = (np.full(wl.d_k, bits[h]) if wl.unit == W.UNIT_HEAD
+                  else bits[h * wl.d_k:(h + 1) * wl.d_k])
+        if np.all(widths == 16):
+            continue
+        r16 = blk[:2 * wl.d_k].view(np.float16).astype(np.float64)
+        c16 = blk[2 * wl.d_k:2 * (wl.d_k + wl.d_v)].view(np.float16).astype(np.float64)
+        for i in range(wl.d_k):
+            if widths[i] == 16:
+                continue
+            step = r16[i] * c16
+            err = np.abs(D[i].astype(np.float64) - S[h, i])
+            exempt = np.zeros(wl.d_v, bool)
+            if wl.n_outliers:
+                exempt = D[i] == np.float16(S[h, i]).astype(np.float32)
+            assert np.all((err <= 0.5 * step * (1 + 2e-3) + 1e-7) | exempt), (h, i)
+
+
+def test_impact_lowers_column_scales_in_the_first_alternation(oracle):
+    """One alternation: lowering rho never lowers a row scale and never raises a column scale
+    (w_i can only shrink); rows with rho = 1 keep their scale."""
+    rng = np.random.default_rng(3)
+    for _ in range(20):
+        S = rng.standard_normal((16, 16)).astype(np.float32)
+        S[rng.integers(0, 16, 4), rng.integers(0, 16, 4)] *= 30
+        qm = rng.choice([1, 7, 31, 127], 16)
+        rho = np.where(rng.random(16) < 0.3, 1.0, rng.uniform(0.05, 1.0, 16)).astype(np.float32)
+        r0, c0 = oracle.fit(S, qm, fit_iters=1)
+        r1, c1 = oracle.fit(S, qm, fit_iters=1, rho=rho)
+        assert np.all(r1 >= r0) and np.all(c1 <= c0)
+        np.testing.assert_array_equal(r1[rho == 1.0], r0[rho == 1.0])
