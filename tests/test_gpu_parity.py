@@ -196,3 +196,24 @@ def test_extreme_gates(name, want_state):
         mis, tot = mis + m, tot + n
     assert mis <= max(1, 1e-4 * tot), (mis, tot)
     assert case.pool.status() == (sq.SQ_OK, 0)
+
+
+def test_empty_batches_are_no_ops():
+    """batch = 0 (and n = 0) on every per-step call: SQ_OK, no launch, no byte changed."""
+    wl = CASES["gdn-s"]
+    case = G.GpuCase(wl)
+    before = case.slots()
+    q, k, v, a, b = case.device_inputs(wl.step_inputs(0))
+    out = torch.empty((wl.batch, wl.n_heads, 4, wl.d_v), dtype=torch.float32, device="cuda")
+    staging = torch.empty((wl.batch, wl.n_heads, wl.d_k, wl.d_v), device="cuda")
+    h, si = case.pool.handle, case.si.data_ptr()
+    ptrs = (q.data_ptr(), k.data_ptr(), v.data_ptr(), a.data_ptr(), b.data_ptr(), out.data_ptr())
+    sq.sq_decode_step(h, si, 0, *ptrs, 0)
+    sq.sq_decode_chunk(h, si, 0, 4, *ptrs, 0)
+    sq.sq_decode_step_split(h, si, 0, *ptrs, staging.data_ptr(), 0, 0)
+    sq.sq_decode_step_split_static(h, si, 0, *ptrs, 0)
+    sq.sq_quantize_fp32_state(h, si, 0, staging.data_ptr(), 0)
+    sq.sq_dequantize_state(h, si, 0, staging.data_ptr(), 0)
+    torch.cuda.synchronize()
+    assert case.pool.status() == (sq.SQ_OK, 0)
+    np.testing.assert_array_equal(case.slots(), before)
