@@ -149,3 +149,24 @@ def test_bad_impacts_rejected(bad):
     imp[1, 3] = bad
     with pytest.raises(sq.SqError):
         case.pool.set_row_impact(imp)
+
+
+def test_weighted_full_size_sampled():
+    """The GDN layer at full size (64 x 32 heads, d = 128) with a row-impact table: two steps,
+    a seeded sample of requests checked against the oracle each time."""
+    wl = W.WORKLOADS["gdn"]
+    imp = impact_of(wl, seed=5)
+    case = weighted_case(wl, imp)
+    sample = np.sort(np.random.default_rng(13).choice(wl.batch, 4, replace=False))
+    for t in range(2):
+        x = wl.step_inputs(t)
+        pre = case.slots()
+        o_gpu, _ = case.step(x)
+        post = case.slots()
+        opool = oracle_pool(wl, imp, pre[case.si_np[sample]])
+        xs = G.sub_inputs(x, sample)
+        o_ref = opool.decode_step(np.arange(sample.size), xs["q"], xs["k"], xs["v"],
+                                  xs["alpha"], xs["beta"])
+        G.close(o_gpu[sample], o_ref, f"step {t} o")
+        G.compare_codes(wl, case.bits, post[case.si_np[sample]],
+                        opool.data.reshape(sample.size, -1), f"step {t}")

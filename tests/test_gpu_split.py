@@ -137,3 +137,24 @@ def test_split_rejects_windowed_pools_and_bad_staging():
     sp.staging = torch.empty(sp.staging.numel() + 1, device="cuda")[1:]  # 4-byte aligned only
     with pytest.raises(sq.SqError):
         sp.step(case.wl.step_inputs(0))
+
+
+def test_split_full_size_sampled():
+    """The split workload at full size (64 requests x 32 heads, d = 128, the launch the bench
+    times): two steps, a seeded sample of requests checked against the oracle each time."""
+    wl = W.WORKLOADS["split"]
+    case = G.GpuCase(wl)
+    sp = Split(case)
+    sample = np.sort(np.random.default_rng(9).choice(wl.batch, 4, replace=False))
+    for t in range(2):
+        x = wl.step_inputs(t)
+        pre = case.slots()
+        o = sp.step(x).cpu().numpy()
+        post = case.slots()
+        opool = G.oracle_pool_from(wl, case.bits, pre[case.si_np[sample]])
+        xs = G.sub_inputs(x, sample)
+        o_ref = opool.decode_step(np.arange(sample.size), xs["q"], xs["k"], xs["v"],
+                                  xs["alpha"], xs["beta"])
+        G.close(o[sample], o_ref, f"step {t} o")
+        G.compare_codes(wl, case.bits, post[case.si_np[sample]],
+                        opool.data.reshape(sample.size, -1), f"step {t}")
