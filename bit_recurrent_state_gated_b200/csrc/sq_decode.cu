@@ -145,23 +145,17 @@ __device__ __forceinline__ void tm_issue(uint32_t taddr, uint32_t (&r)[16]) {
         "=r"(r[14]), "=r"(r[15])
       : "r"(taddr));
 }
-// Wait for every load this thread issued, then hand the registers of `r` over as 8 pairs (the
-// registers are inputs of the same statement as the wait, so nothing reads them earlier).
-__device__ __forceinline__ void tm_take(const uint32_t (&r)[16], float2 (&v)[8]) {
-  uint64_t u[8];
-  asm volatile(
-      "tcgen05.wait::ld.sync.aligned;\n\t"
-      "mov.b64 %0, {%8,%9};\n\tmov.b64 %1, {%10,%11};\n\tmov.b64 %2, {%12,%13};\n\t"
-      "mov.b64 %3, {%14,%15};\n\tmov.b64 %4, {%16,%17};\n\tmov.b64 %5, {%18,%19};\n\t"
-      "mov.b64 %6, {%20,%21};\n\tmov.b64 %7, {%22,%23};"
-      : "=l"(u[0]), "=l"(u[1]), "=l"(u[2]), "=l"(u[3]), "=l"(u[4]), "=l"(u[5]), "=l"(u[6]),
-        "=l"(u[7])
-      : "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
-        "r"(r[15])
-      : "memory");
+// Wait for every load this thread issued; the registers are operands of the wait, so nothing
+// reads them earlier. Then view them as 8 pairs.
+__device__ __forceinline__ void tm_take(uint32_t (&r)[16], float2 (&v)[8]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                 "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                 "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
+               :
+               : "memory");
 #pragma unroll
-  for (int e = 0; e < 8; ++e) v[e] = *reinterpret_cast<const float2*>(&u[e]);
+  for (int e = 0; e < 8; ++e) v[e] = make_float2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]));
 }
 
 // Run body(ch, v) over chunks 0..nch-1 (nch even) of the thread's tile, each chunk's load in
