@@ -11,9 +11,10 @@
  * Conventions for every call
  *   - Pointers marked (device) are CUDA device pointers; (host) are ordinary host pointers.
  *     Device pointers must be 16-byte aligned; the pool buffer must be 256-byte aligned.
- *   - The caller owns every buffer it passes. The pool handle owns only its host metadata and
- *     a few small device tables (offset tables and a status word), allocated at create and
- *     freed at destroy.
+ *   - The caller owns every buffer it passes. The pool handle owns only its host metadata, a
+ *     few small device tables (offset tables and a status word, allocated at create; the row
+ *     impact table, allocated by sq_pool_set_row_impact) and, after its first split step, two
+ *     CUDA events; destroy frees them all.
  *   - `stream` is a cudaStream_t passed as void*; NULL means the legacy default stream. Calls
  *     that take a stream only enqueue work and return; they do not synchronize.
  *   - Every call returns an sq_status. Nothing aborts, traps or prints. Argument errors are
@@ -22,7 +23,8 @@
  *     device status word, and the affected (request, head) is skipped: its slot bytes stay as
  *     they were and its output row is filled with NaN. sq_pool_status() reads and clears it.
  *   - Within one call every slot index must be distinct; duplicates are not detected and give
- *     an undefined result. Calls on one pool must not overlap in time on different streams.
+ *     an undefined result. Calls on one pool must not overlap in time on different streams
+ *     (the second stream of sq_decode_step_split is ordered by the pool itself).
  *   - State layout: S[i][j] with i the key channel ("key row", [SQ-E] fitting paragraph) and
  *     j the value channel ("value column", [SQ-N]). Dense fp32 states are row-major
  *     [n][n_heads][d_k][d_v].
