@@ -188,33 +188,50 @@ class ClockSampler:
 
 # ---- CPU oracle (baseline and reference arm) ----------------------------------------------------
 
+class OracleSample:
+    """A bounded sample of the workload for the CPU oracle: the first few requests of the batch
+    (all heads) in an oracle pool, with a few steps of inputs, stepped on demand."""
+
+    def __init__(self, wl: W.Workload, t0: int = 0):
+        import oracle
+        self.threads = oracle.default_threads()
+        self.n_req = max(1, min(wl.batch, self.threads))
+        # a chunk of T tokens is the windowed oracle with W = T (requantized after the T-th token)
+        window = wl.tokens if wl.tokens > 1 else wl.window
+        lay = oracle.Layout(wl.n_heads, wl.d_k, wl.d_v, wl.unit, wl.gate, wl.fit_iters, window,
+                            wl.n_outliers)
+        self.pool = oracle.Pool(lay, wl.bits(), self.n_req)
+        self.step = self.pool.window_step if window > 1 else self.pool.decode_step
+        self.si = np.arange(self.n_req, dtype=np.int32)
+        self.pool.quantize(self.si, wl.initial_state(wl.slot_idx()[:self.n_req]))
+        self.sets = []
+        for t in range(t0, t0 + max(4, wl.tokens)):
+            x = wl.step_inputs(t)
+            self.sets.append({k: np.ascontiguousarray(v[:self.n_req]) for k, v in x.items()})
+        self.calls = 0
+
+    def run(self, seconds: float):
+        """Step until `seconds` of oracle time (at least one call): (request-steps, seconds)."""
+        done, busy = 0, 0.0
+        while busy < seconds or done == 0:  # only the oracle's own calls are timed
+            xs = self.sets[self.calls % len(self.sets)]
+            ts = time.perf_counter()
+            self.step(self.si, xs["q"], xs["k"], xs["v"], xs["alpha"], xs["beta"],
+                      threads=self.threads)
+            busy += time.perf_counter() - ts
+            done += self.n_req
+            self.calls += 1
+        return done, busy
+
+    def describe(self, wl: W.Workload) -> str:
+        return f"{self.n_req} requests x {wl.n_heads} heads"
+
+
 def oracle_rate(wl: W.Workload, seconds: float, t0: int = 0):
-    """Request-steps/s of the CPU oracle on a bounded sample of the workload: the first few
-    requests of the batch (all heads), stepped repeatedly until `seconds` of CPU time."""
-    import oracle
-    threads = oracle.default_threads()
-    n_req = max(1, min(wl.batch, threads))
-    # a chunk of T tokens is the windowed oracle with W = T (requantized after the T-th token)
-    window = wl.tokens if wl.tokens > 1 else wl.window
-    lay = oracle.Layout(wl.n_heads, wl.d_k, wl.d_v, wl.unit, wl.gate, wl.fit_iters, window,
-                        wl.n_outliers)
-    pool = oracle.Pool(lay, wl.bits(), n_req)
-    step = pool.window_step if window > 1 else pool.decode_step
-    si = np.arange(n_req, dtype=np.int32)
-    pool.quantize(si, wl.initial_state(wl.slot_idx()[:n_req]))
-    sets = []
-    for t in range(t0, t0 + max(4, wl.tokens)):
-        x = wl.step_inputs(t)
-        sets.append({k: np.ascontiguousarray(v[:n_req]) for k, v in x.items()})
-    done, busy, n = 0, 0.0, 0
-    while busy < seconds:  # only the oracle's own calls are timed
-        xs = sets[n % len(sets)]
-        ts = time.perf_counter()
-        step(si, xs["q"], xs["k"], xs["v"], xs["alpha"], xs["beta"], threads=threads)
-        busy += time.perf_counter() - ts
-        done += n_req
-        n += 1
-    return done / busy, threads, f"{n_req} requests x {wl.n_heads} heads, {n} steps"
+    """Request-steps/s of the CPU oracle on a bounded sample of the workload."""
+    sample = OracleSample(wl, t0)
+    done, busy = sample.run(seconds)
+    return done / busy, sample.threads, f"{sample.describe(wl)}, {sample.calls} steps"
 
 
 # ---- GPU arm -----------------------------------------------------------------------------------
@@ -460,16 +477,20 @@ def run_reference(args, info):
     if info.rank != 0:
         return None
     wl = W.WORKLOADS[args.workload]
-    per_step = max(0.5, min(args.cpu_seconds, 150.0 / max(1, args.steps + args.warmup)))
-    for t in range(args.warmup):
-        oracle_rate(wl, per_step / 4, t0=t)
-    rates, cores, sample = [], 0, ""
+    # every step a bounded sample, sized so the whole run stays within about 150 s of oracle time
+    per_step = max(0.02, min(args.cpu_seconds, 150.0 / max(1, args.steps + args.warmup)))
+    sample = OracleSample(wl)
+    for _ in range(args.warmup):
+        sample.run(per_step)
+    done = busy = 0.0
     t0 = time.perf_counter()
-    for t in range(args.steps):
-        r, cores, sample = oracle_rate(wl, per_step, t0=args.warmup + t)
-        rates.append(r)
+    for _ in range(args.steps):
+        d, b = sample.run(per_step)
+        done, busy = done + d, busy + b
     el = time.perf_counter() - t0
-    value = statistics.mean(rates)
+    value = done / busy
+    cores = sample.threads
+    sample_txt = f"{sample.describe(wl)}, about {per_step:.3g} s of oracle time"
     return {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
         "n_gpus": info.world, "steps": args.steps, "warmup": args.warmup,
@@ -479,7 +500,7 @@ def run_reference(args, info):
         "config": {"workload": f"{wl.name}: {wl.notes}", "batch_per_gpu": wl.batch,
                    "heads": wl.n_heads, "d_k": wl.d_k, "d_v": wl.d_v},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": f"per step: {sample}"},
+                         "sample": f"per step: {sample_txt}"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
