@@ -1263,8 +1263,13 @@ __device__ __forceinline__ void window_fold(const Ctx<FULL>& c, const StepArgs& 
       }
     });
     __syncthreads();
+    // The thread maxima can exceed the tile's current values (an element changed by a frozen
+    // entry's patch after its maximum was taken), so the threshold may lie above the n-th
+    // largest element; then fewer than n candidates exist and the exact path below decides.
+    // With n or more candidates every element of the top n is among them.
     const int nc = misc[0];
-    if (nc <= kMaxCand) {
+    const bool ranked = nc >= n_out && nc <= kMaxCand;
+    if (ranked) {
       // rank of each candidate by (|v| desc, flat index asc); the first n go to the stage
       // arrays in that order, then to oidx/opos/oval in ascending flat index
       int* sidx = sp<int>(W_CSEL);
@@ -1293,7 +1298,7 @@ __device__ __forceinline__ void window_fold(const Ctx<FULL>& c, const StepArgs& 
         opos[rank] = spos[tid];
         oval[rank] = sval[tid];
       }
-    } else {  // many equal values: n rounds of an exact arg-max over the tile
+    } else {  // many equal values, or too few candidates: n rounds of an exact arg-max
       for (int r = 0; r < n_out; ++r) {
         unsigned long long best = 0;
         int bp = 0;
@@ -1342,7 +1347,7 @@ __device__ __forceinline__ void window_fold(const Ctx<FULL>& c, const StepArgs& 
       }
     }
     __syncthreads();
-    if (nc > kMaxCand && tid == 0) {  // fallback path: ascending flat index
+    if (!ranked && tid == 0) {  // exact path: ascending flat index
       for (int x = 1; x < n_out; ++x) {
         const int ki = oidx[x], kp = opos[x];
         const float kv = oval[x];
