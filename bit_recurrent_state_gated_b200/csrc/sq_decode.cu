@@ -28,10 +28,10 @@
 // bulk copies issued right after the current item's first barrier, when the single staging
 // buffer is free again.
 //
-// Arithmetic: the refit follows the oracle's rule step for step with correctly rounded
-// operations (r_i = max(m_i / Q_i, 2^-14), w_i = 1/(r_i Q_i), c_j = max(max_i |S_ij| w_i,
-// 2^-14), v_j = 1/c_j, fp16 rounding once); the code multipliers 1/r16 and 1/c16 are correctly
-// rounded as well. Codes need no clamp: the fit makes every |S_ij| w_i <= c_j, so the quotient
+// Arithmetic: the refit follows the oracle's rule step for step: r_i = max(m_i / Q_i, 2^-14)
+// correctly rounded, c_j = max(max_i |S_ij| w_i, 2^-14), fp16 rounding once; w_i = 1/(r_i Q_i)
+// and v_j = 1/c_j use the hardware's approximate reciprocal, the code multipliers 1/r16 and
+// 1/c16 are correctly rounded. Codes need no clamp: every |S_ij| w_i <= c_j, so the quotient
 // S_ij / (r16_i c16_j) is at most Q (1 + 2^-10) in magnitude, less than Q + 1/2 for Q <= 127.
 // The state is the GPU's own fp32 update (fused multiply-adds), so its scales and codes are
 // compared with the oracle's within the stated agreement.
