@@ -26,7 +26,7 @@ class OracleError(RuntimeError):
 class _Layout(C.Structure):
     _fields_ = [(n, C.c_int32) for n in
                 ("n_heads", "d_k", "d_v", "unit", "gate", "fit_iters", "window", "n_outliers")
-                ] + [("rho", C.c_void_p)]
+                ] + [("omega", C.c_void_p)]
 
 
 @dataclass(frozen=True)
@@ -41,21 +41,19 @@ class Layout:
     n_outliers: int = 0
     row_impact: object = field(default=None, compare=False, hash=False)  # [n_heads][d_k] > 0
 
-    def rho(self):
-        """Impact scores divided by the largest of their head (fp64 division, then fp32)."""
+    def omega(self):
+        """Column-pass weights of the impact-weighted fit (orc_impact_weights), or None."""
         if self.row_impact is None:
             return None
-        imp = np.asarray(self.row_impact, dtype=np.float64).reshape(self.n_heads, self.d_k)
-        assert np.all(np.isfinite(imp)) and np.all(imp > 0)
-        return np.ascontiguousarray((imp / imp.max(axis=1, keepdims=True)).astype(np.float32))
+        return impact_weights(self.row_impact, self.n_heads, self.d_k)
 
     def c(self) -> _Layout:
         lay = _Layout(self.n_heads, self.d_k, self.d_v, self.unit, self.gate, self.fit_iters,
                       self.window, self.n_outliers, None)
-        rho = self.rho()
-        if rho is not None:
-            lay.rho = rho.ctypes.data
-            lay.keep = rho  # the table lives as long as the structure
+        om = self.omega()
+        if om is not None:
+            lay.omega = om.ctypes.data
+            lay.keep = om  # the table lives as long as the structure
         return lay
 
     @property
@@ -82,6 +80,7 @@ def lib():
             "orc_f32_to_f16_bits": [C.c_float],
             "orc_f16_bits_to_f32": [C.c_uint16],
             "orc_fit": [C.c_int, C.c_int, C.c_int, P, P, P, P, P, P],
+            "orc_impact_weights": [C.c_int, C.c_int, P, P],
             "orc_select_outliers": [C.c_int, C.c_int, P, P, C.c_int, P],
             "orc_quantize_head": [P, P, C.c_int, P, P],
             "orc_dequantize_head": [P, P, C.c_int, P, P],
@@ -163,18 +162,26 @@ def f32_to_f16_bits(x: float) -> int:
     return int(lib().orc_f32_to_f16_bits(float(x)))
 
 
-def fit(S: np.ndarray, qmax, fit_iters: int = 2, excluded=None, rho=None):
-    """(r, c) of the dual-axis fit; rho: optional per-row weights in (0, 1] (impact)."""
+def fit(S: np.ndarray, qmax, fit_iters: int = 2, excluded=None, omega=None):
+    """(r, c) of the dual-axis fit; omega: optional per-row column-pass weights in (0, 1]."""
     S = np.ascontiguousarray(S, dtype=np.float32)
     dk, dv = S.shape
     q = np.ascontiguousarray(np.asarray(qmax, dtype=np.int32))
     ex = None if excluded is None else np.ascontiguousarray(np.asarray(excluded, dtype=np.uint8))
-    rh = None if rho is None else np.ascontiguousarray(np.asarray(rho, dtype=np.float32))
+    om = None if omega is None else np.ascontiguousarray(np.asarray(omega, dtype=np.float32))
     r = np.zeros(dk, dtype=np.float32)
     c = np.zeros(dv, dtype=np.float32)
     _chk(lib().orc_fit(dk, dv, fit_iters, _p(S), _p(q), None if ex is None else _p(ex),
-                       None if rh is None else _p(rh), _p(r), _p(c)), "fit")
+                       None if om is None else _p(om), _p(r), _p(c)), "fit")
     return r, c
+
+
+def impact_weights(impact, n_heads: int, d_k: int) -> np.ndarray:
+    """Column-pass weights [n_heads][d_k] of the impact-weighted fit from row impact scores."""
+    imp = np.ascontiguousarray(np.asarray(impact, dtype=np.float32).reshape(n_heads, d_k))
+    om = np.zeros((n_heads, d_k), dtype=np.float32)
+    _chk(lib().orc_impact_weights(n_heads, d_k, _p(imp), _p(om)), "impact_weights")
+    return om
 
 
 def select_outliers(S: np.ndarray, qmax, n: int) -> np.ndarray:

@@ -26,10 +26,11 @@
  * Parity pins (tests/test_oracle_pins.py) cover every exported function: closed forms of the
  * delta rule, Proposition 1, quantize/dequantize idempotence, the half-step error bound, the
  * textbook special cases, brute force on 4x4 tiles, and a format-size check against the
- * compression ratios [SQ-E] prints. One part is "parity unpinned": the row-impact weighting
- * of orc_fit (rho != NULL), whose formula the pages do not print; the reading taken is pinned
- * only by its special cases (a hand-worked 2 x 2 example, rho = 1 giving the plain fit, codes
- * within [-Q, Q] and the half-step bound, monotone first alternation).
+ * compression ratios [SQ-E] prints. The row-impact weighting of orc_fit (omega != NULL),
+ * whose formula the pages do not print, is pinned by its stated purpose (a lower
+ * impact-weighted reconstruction error than the plain fit on seeded heads) and its special
+ * cases (a hand-worked 2 x 2 example, equal impacts giving the plain fit, codes within [-Q, Q]
+ * and the half-step bound, monotone first alternation).
  */
 #include "sq_oracle.h"
 
@@ -169,19 +170,20 @@ void orc_unpack_row(int b, int n, const uint8_t* in, int32_t* u) {
  * Rows with qmax[i] == 0 (fp16 pivot rows) and elements with excluded[] set (outliers) take
  * no part. The caller rounds r and c to fp16 once, at the end.
  *
- * Impact weighting (rho != NULL; parity unpinned beyond its special cases, the pages print no
- * formula). [SQ-E] experimental-setup paragraph: the row scale weighs the row's current size
- * together with its impact score, and the column scale penalizes reconstruction error more in
- * high-impact rows (wide range for large rows, finer resolution for important rows). Reading
- * taken: with rho_i in (0, 1] the row's impact divided by the largest of its head,
- *     r_i = max( fl(q_i / rho_i) capped at 65504 , q_i , 2^-14 ),  q_i = fl(m_i / Q_i),
- * so a low-impact row takes a wider step than its own range needs, its w_i shrinks, and the
- * column maxima c_j are set by the high-impact rows. No element leaves [-Q, Q] (every
- * |S_ij| w_i <= c_j still holds), rho = 1 is the plain fit above, and scaling every rho_i of a
- * head by one factor leaves r_i c_j unchanged up to rounding.
+ * Impact weighting (omega != NULL; the pages print no formula). [SQ-E] experimental-setup
+ * paragraph: the row scale weighs the row's current size together with its impact score, and
+ * the column scale penalizes reconstruction error more in high-impact rows (wide range for
+ * large rows, finer resolution for important rows). Reading taken: every row pass stays as
+ * above (each row's scale follows its own size), and the column pass counts row i with a
+ * weight omega_i in (0, 1], w_i = fl(omega_i * fl(1 / fl(r_i * Q_i))) (omega_i = 1: the plain
+ * w_i), so the column scales follow the high-impact rows; after the last alternation every
+ * row with omega_i < 1 is fit once more against the final column scales,
+ *     r_i = max( r_i , fl( max_j fl(|S_ij| * fl(1/c_j)) / Q_i ) ),
+ * so no element of it leaves [-Q, Q]. The weights come from orc_impact_weights. omega = 1
+ * everywhere is the plain fit bit for bit.
  * ---------------------------------------------------------------------------------------- */
 int orc_fit(int d_k, int d_v, int fit_iters, const float* S, const int32_t* qmax,
-            const uint8_t* excluded, const float* rho, float* r, float* c) {
+            const uint8_t* excluded, const float* omega, float* r, float* c) {
   float* inv_c = (float*)malloc(sizeof(float) * (size_t)d_v);
   float* w = (float*)malloc(sizeof(float) * (size_t)d_k);
   if (!inv_c || !w) {
@@ -206,15 +208,12 @@ int orc_fit(int d_k, int d_v, int fit_iters, const float* S, const int32_t* qmax
         if (a > m) m = a;
       }
       float ri = m / (float)qmax[i];
-      float rr = ri > ORC_SCALE_FLOOR ? ri : ORC_SCALE_FLOOR;
-      if (rho) {
-        float wide = ri / rho[i];
-        if (wide > 65504.0f) wide = 65504.0f;
-        if (wide > rr) rr = wide;
-      }
-      r[i] = rr;
+      r[i] = ri > ORC_SCALE_FLOOR ? ri : ORC_SCALE_FLOOR;
     }
-    for (int i = 0; i < d_k; ++i) w[i] = qmax[i] ? 1.0f / (r[i] * (float)qmax[i]) : 0.0f;
+    for (int i = 0; i < d_k; ++i) {
+      w[i] = qmax[i] ? 1.0f / (r[i] * (float)qmax[i]) : 0.0f;
+      if (omega && omega[i] < 1.0f) w[i] = omega[i] * w[i];
+    }
     for (int j = 0; j < d_v; ++j) { /* column pass */
       float m = 0.0f;
       for (int i = 0; i < d_k; ++i) {
@@ -227,8 +226,49 @@ int orc_fit(int d_k, int d_v, int fit_iters, const float* S, const int32_t* qmax
       inv_c[j] = 1.0f / c[j];
     }
   }
+  if (omega) { /* rows counted with omega < 1: fit once more against the final column scales */
+    for (int i = 0; i < d_k; ++i) {
+      if (qmax[i] == 0 || !(omega[i] < 1.0f)) continue;
+      float m = 0.0f;
+      for (int j = 0; j < d_v; ++j) {
+        if (excluded && excluded[(size_t)i * d_v + j]) continue;
+        float a = fabsf(S[(size_t)i * d_v + j]) * inv_c[j];
+        if (a > m) m = a;
+      }
+      float ri = m / (float)qmax[i];
+      if (ri > r[i]) r[i] = ri;
+    }
+  }
   free(inv_c);
   free(w);
+  return ORC_OK;
+}
+
+/* ------------------------------------------------------------------------------------------
+ * Column-pass weights of the impact-weighted fit (reading of [SQ-E] experimental-setup
+ * paragraph; see orc_fit). A quantization step of r_i c_j costs row i an error that grows with
+ * (r_i c_j)^2, weighted by its impact. Lowering a column scale c_j refines that column in every
+ * row, but the row that sets it (its "anchor") must widen its own scale r_i by the same factor
+ * f to keep its codes in range. With d_v columns of similar scale, the gain is about
+ * (1 - 1/f^2) times the head's mean weighted row error and the cost f^2 - 1 times the anchor's,
+ * so the lowering pays while f^2 < mean impact / impact_i. The column pass therefore counts
+ * row i with weight 1 / f = min(1, sqrt(impact_i / mean impact of its head)), in fp64, rounded
+ * to fp32 once. impact: [n_heads][d_k], every entry > 0 and finite. Equal impacts give 1.
+ * ---------------------------------------------------------------------------------------- */
+int orc_impact_weights(int n_heads, int d_k, const float* impact, float* omega) {
+  for (int h = 0; h < n_heads; ++h) {
+    const float* im = impact + (size_t)h * d_k;
+    double sum = 0.0;
+    for (int i = 0; i < d_k; ++i) {
+      if (!(im[i] > 0.0f) || !isfinite(im[i])) return ORC_ERR_ARG;
+      sum += (double)im[i];
+    }
+    const double mean = sum / (double)d_k;
+    for (int i = 0; i < d_k; ++i) {
+      double x = sqrt((double)im[i] / mean);
+      omega[(size_t)h * d_k + i] = (float)(x < 1.0 ? x : 1.0);
+    }
+  }
   return ORC_OK;
 }
 
@@ -323,7 +363,7 @@ int orc_quantize_head(const orc_layout* L, const uint8_t* bits, int h, const flo
     if (st) goto done;
     for (int t = 0; t < L->n_outliers; ++t) excl[oidx[t]] = 1;
   }
-  orc_fit(dk, dv, L->fit_iters, S, qmax, excl, L->rho ? L->rho + (size_t)h * dk : NULL, r, c);
+  orc_fit(dk, dv, L->fit_iters, S, qmax, excl, L->omega ? L->omega + (size_t)h * dk : NULL, r, c);
 
   uint8_t* r16p = block;
   uint8_t* c16p = block + 2 * (size_t)dk;

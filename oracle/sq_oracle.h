@@ -12,7 +12,7 @@
  *   LeapQuant news        = "LeapQuant、線形注意の推論を1.47倍高速化", news.affectosphere.group
  *
  * Parity status of each function is listed at the top of sq_oracle.c: the row-impact
- * weighting of orc_fit (orc_layout.rho) is "parity unpinned" beyond its special cases.
+ * weighting of orc_fit (orc_layout.omega) is pinned by its stated purpose and special cases.
  */
 #ifndef SQ_ORACLE_H
 #define SQ_ORACLE_H
@@ -34,8 +34,8 @@ typedef struct {
   int32_t fit_iters;  /* alternations of the row/column max-abs fit (>= 1) */
   int32_t window;     /* 1: requantize after every step; W > 1: after every W steps */
   int32_t n_outliers; /* entries per head kept in fp16 at each requantization */
-  const float* rho;   /* NULL, or per key row of each head [n_heads][d_k]: the row's impact
-                         score divided by the largest of its head (orc_fit) */
+  const float* omega; /* NULL, or per key row of each head [n_heads][d_k]: the row's weight
+                         in the column pass of the fit (orc_impact_weights, orc_fit) */
 } orc_layout;
 
 /* ---- format ---- */
@@ -50,7 +50,8 @@ float orc_f16_bits_to_f32(uint16_t h);
 
 /* ---- one head ---- */
 int orc_fit(int d_k, int d_v, int fit_iters, const float* S, const int32_t* qmax,
-            const uint8_t* excluded, const float* rho, float* r, float* c);
+            const uint8_t* excluded, const float* omega, float* r, float* c);
+int orc_impact_weights(int n_heads, int d_k, const float* impact, float* omega);
 int orc_select_outliers(int d_k, int d_v, const float* S, const int32_t* qmax, int n,
                         int32_t* idx_out);
 int orc_quantize_head(const orc_layout* L, const uint8_t* bits, int h, const float* S,

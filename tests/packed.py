@@ -2,9 +2,11 @@
 
 Splits a pool's bytes into fp16 scales, integer codes and fp16 pivot / outlier values, so
 parity tests can compare codes element by element. It follows the format as the header
-include/sq.h states it and uses only numpy bit unpacking.
+include/sq.h states it and uses only numpy shifts and masks.
 """
 from __future__ import annotations
+
+from functools import lru_cache
 
 import numpy as np
 
@@ -15,48 +17,87 @@ def _widths(unit: int, bits: np.ndarray, H: int, dk: int) -> np.ndarray:
     return np.asarray(bits, np.int64).reshape(H, dk)
 
 
+def _plan(unit: int, bits, H: int, dk: int, dv: int, n_outliers: int):
+    return _plan_cached(unit, np.asarray(bits, np.uint8).tobytes(), H, dk, dv, n_outliers)
+
+
+@lru_cache(maxsize=32)
+def _plan_cached(unit: int, bits_bytes: bytes, H: int, dk: int, dv: int, n_outliers: int):
+    """Byte offsets of every head block and row, as the format in include/sq.h lays them out."""
+    W = _widths(unit, np.frombuffer(bits_bytes, np.uint8), H, dk)
+    row_off = np.zeros((H, dk), np.int64)
+    head_off = np.zeros(H, np.int64)
+    out_off = np.zeros(H, np.int64)
+    off = 0
+    for h in range(H):
+        head_off[h] = off
+        if unit == 0 and W[h, 0] == 16:
+            size = 2 * dk * dv
+        else:
+            p = off + 2 * (dk + dv)
+            for i in range(dk):
+                row_off[h, i] = p
+                p += dv * int(W[h, i]) // 8
+            out_off[h] = p
+            size = p + 4 * n_outliers - off
+        off += (size + 15) // 16 * 16
+    return W, row_off, head_off, out_off
+
+
+def _fields(raw: np.ndarray, b: int, dv: int) -> np.ndarray:
+    """The dv b-bit fields of each row of raw [..., dv * b / 8] (uint8), LSB first: field j
+    sits at bits [j b, (j + 1) b) of the row's little-endian bit stream."""
+    x = raw.astype(np.int64)
+    if b == 8:
+        return x
+    if b == 6:  # three bytes hold four fields
+        g = x.reshape(*x.shape[:-1], dv // 4, 3)
+        word = g[..., 0] | (g[..., 1] << 8) | (g[..., 2] << 16)
+        return ((word[..., None] >> (6 * np.arange(4))) & 63).reshape(*x.shape[:-1], dv)
+    per = 8 // b  # fields per byte
+    return ((x[..., None] >> (b * np.arange(per))) & ((1 << b) - 1)).reshape(*x.shape[:-1], dv)
+
+
 def decode(slots: np.ndarray, unit: int, bits, H: int, dk: int, dv: int, n_outliers: int = 0):
     """slots: uint8 [n, slot_bytes]. Returns dict of arrays over [n, H, ...]:
     codes int64 [n,H,dk,dv] (0 on fp16 rows), f16 float32 [n,H,dk,dv] (fp16 values on pivot
     rows / heads, outliers, else 0), r16/c16 float64, pivot bool [H,dk], out_idx/out_val."""
     n = slots.shape[0]
-    W = _widths(unit, bits, H, dk)
+    W, row_off, head_off, out_off = _plan(unit, bits, H, dk, dv, n_outliers)
     codes = np.zeros((n, H, dk, dv), np.int64)
     f16 = np.zeros((n, H, dk, dv), np.float32)
     r16 = np.zeros((n, H, dk))
     c16 = np.ones((n, H, dv))
     outliers = np.zeros((n, H, n_outliers), np.int64)
-    off = 0
     for h in range(H):
-        pivot_head = unit == 0 and W[h, 0] == 16
-        start = off
-        if pivot_head:
+        off = head_off[h]
+        if unit == 0 and W[h, 0] == 16:
             blk = slots[:, off:off + 2 * dk * dv]
             f16[:, h] = blk.copy().view(np.float16).reshape(n, dk, dv).astype(np.float32)
-            size = 2 * dk * dv
         else:
             r16[:, h] = slots[:, off:off + 2 * dk].copy().view(np.float16).astype(np.float64)
-            c16[:, h] = slots[:, off + 2 * dk:off + 2 * dk + 2 * dv].copy().view(
+            c16[:, h] = slots[:, off + 2 * dk:off + 2 * (dk + dv)].copy().view(
                 np.float16).astype(np.float64)
-            p = off + 2 * (dk + dv)
-            for i in range(dk):
-                b = int(W[h, i])
-                nb = dv * b // 8
-                raw = slots[:, p:p + nb]
-                if b == 16:
-                    f16[:, h, i] = raw.copy().view(np.float16).astype(np.float32)
-                else:
-                    bitsarr = np.unpackbits(raw, axis=1, bitorder="little")[:, :dv * b]
-                    u = (bitsarr.reshape(n, dv, b).astype(np.int64) << np.arange(b)).sum(-1)
-                    codes[:, h, i] = u - (1 << (b - 1))
-                p += nb
-            for t in range(n_outliers):
-                idx = slots[:, p + 4 * t:p + 4 * t + 2].copy().view(np.uint16)[:, 0].astype(np.int64)
-                val = slots[:, p + 4 * t + 2:p + 4 * t + 4].copy().view(np.float16)[:, 0]
-                outliers[:, h, t] = idx
-                f16[np.arange(n), h, idx // dv, idx % dv] = val.astype(np.float32)
-            size = p + 4 * n_outliers - off
-        off = start + (size + 15) // 16 * 16
+    quant_rows = ~((W == 16) & (np.asarray([unit == 0] * H)[:, None]))
+    for b in (2, 4, 6, 8, 16):  # all rows of one width at once
+        hs, rs = np.nonzero((W == b) & quant_rows)
+        if hs.size == 0:
+            continue
+        nb = dv * b // 8
+        raw = slots[:, row_off[hs, rs][:, None] + np.arange(nb)[None, :]]  # [n, rows, nb]
+        if b == 16:
+            f16[:, hs, rs] = raw.copy().view(np.float16).astype(np.float32)
+        else:
+            codes[:, hs, rs] = _fields(raw, b, dv) - (1 << (b - 1))
+    for h in range(H):
+        if unit == 0 and W[h, 0] == 16:
+            continue
+        p = out_off[h]
+        for t in range(n_outliers):
+            idx = slots[:, p + 4 * t:p + 4 * t + 2].copy().view(np.uint16)[:, 0].astype(np.int64)
+            val = slots[:, p + 4 * t + 2:p + 4 * t + 4].copy().view(np.float16)[:, 0]
+            outliers[:, h, t] = idx
+            f16[np.arange(n), h, idx // dv, idx % dv] = val.astype(np.float32)
     pivot = W == 16
     return dict(codes=codes, f16=f16, r16=r16, c16=c16, pivot=pivot, outliers=outliers,
                 widths=W)
