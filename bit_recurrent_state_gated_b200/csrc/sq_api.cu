@@ -27,11 +27,14 @@ struct sq_pool {
   int32_t* d_order = nullptr;
   int32_t* d_flag = nullptr;
   int device = 0, num_sms = 0;
-  float* d_rho = nullptr;  // row impact weights [H][d_k] (sq_pool_set_row_impact)
-  bool has_rho = false;
+  float* d_omega = nullptr;  // column-pass weights [H][d_k] (sq_pool_set_row_impact)
+  bool has_omega = false;
   // side-stream split: the last split's requantization, which later calls on the pool wait for
   cudaEvent_t ev_update = nullptr, ev_side = nullptr;
   bool side_pending = false;
+  // bounded waits of the decode kernel (sq_debug_set_wait)
+  uint64_t wait_ns = 1000000000ull;
+  uint32_t extra_tx = 0;
 };
 
 namespace sq {
@@ -187,7 +190,9 @@ sq::StepArgs step_args(sq_pool* p, const int32_t* slot_idx, int32_t batch, const
   a.side_head_bytes = (int64_t)p->side_head_bytes;
   a.window = p->L.window;
   a.n_outliers = p->L.n_outliers;
-  a.rho = p->has_rho ? p->d_rho : nullptr;
+  a.omega = p->has_omega ? p->d_omega : nullptr;
+  a.wait_ns = p->wait_ns;
+  a.extra_tx = p->extra_tx;
   return a;
 }
 
@@ -213,7 +218,7 @@ sq::QuantArgs quant_args(sq_pool* p, const int32_t* slot_idx, int32_t n, const f
   a.side = p->side_slot_bytes ? p->base + (size_t)p->L.n_slots * p->slot_bytes : nullptr;
   a.side_slot_bytes = (int64_t)p->side_slot_bytes;
   a.side_head_bytes = (int64_t)p->side_head_bytes;
-  a.rho = p->has_rho ? p->d_rho : nullptr;
+  a.omega = p->has_omega ? p->d_omega : nullptr;
   return a;
 }
 
@@ -310,7 +315,7 @@ sq_status sq_state_pool_destroy(sq_pool* pool) {
   cudaFree(pool->d_srows);
   cudaFree(pool->d_flag);
   cudaFree(pool->d_order);
-  cudaFree(pool->d_rho);
+  cudaFree(pool->d_omega);
   if (pool->ev_update) cudaEventDestroy(pool->ev_update);
   if (pool->ev_side) cudaEventDestroy(pool->ev_side);
   delete pool;
@@ -432,28 +437,36 @@ sq_status sq_window_flush(sq_pool* pool, const int32_t* slot_idx, int32_t n, voi
 sq_status sq_pool_set_row_impact(sq_pool* pool, const float* impact) {
   if (!pool) return SQ_ERR_INVALID_ARG;
   if (!impact) {
-    pool->has_rho = false;
+    pool->has_omega = false;
     return SQ_OK;
   }
+  // Weight of row i in the column passes of the fit: min(1, sqrt(impact_i / mean impact of its
+  // head)), in double precision, rounded to fp32 once. Lowering a column scale refines that
+  // column in every row but widens the row that sets it; with d_v columns of similar scale the
+  // trade pays while the widening factor f satisfies f^2 < mean impact / impact_i, so the row
+  // counts with 1 / f. Equal impacts give 1 everywhere: the plain fit.
   const int H = pool->L.n_heads, dk = pool->L.d_k;
-  std::vector<float> rho((size_t)H * dk);
+  std::vector<float> omega((size_t)H * dk);
   for (int h = 0; h < H; ++h) {
-    double mx = 0.0;
+    double sum = 0.0;
     for (int i = 0; i < dk; ++i) {
       const double x = impact[(size_t)h * dk + i];
       if (!(x > 0.0) || !std::isfinite(x)) return SQ_ERR_INVALID_ARG;
-      mx = x > mx ? x : mx;
+      sum += x;
     }
-    for (int i = 0; i < dk; ++i)
-      rho[(size_t)h * dk + i] = (float)((double)impact[(size_t)h * dk + i] / mx);
+    const double mean = sum / dk;
+    for (int i = 0; i < dk; ++i) {
+      const double x = std::sqrt((double)impact[(size_t)h * dk + i] / mean);
+      omega[(size_t)h * dk + i] = (float)(x < 1.0 ? x : 1.0);
+    }
   }
   cudaError_t e = cudaDeviceSynchronize();  // no kernel of this pool may still read the table
-  if (e == cudaSuccess && !pool->d_rho)
-    e = cudaMalloc(&pool->d_rho, rho.size() * sizeof(float));
+  if (e == cudaSuccess && !pool->d_omega)
+    e = cudaMalloc(&pool->d_omega, omega.size() * sizeof(float));
   if (e == cudaSuccess)
-    e = cudaMemcpy(pool->d_rho, rho.data(), rho.size() * sizeof(float), cudaMemcpyHostToDevice);
+    e = cudaMemcpy(pool->d_omega, omega.data(), omega.size() * sizeof(float), cudaMemcpyHostToDevice);
   if (e != cudaSuccess) return cuda_status(e);
-  pool->has_rho = true;
+  pool->has_omega = true;
   return SQ_OK;
 }
 
@@ -467,6 +480,13 @@ sq_status sq_pool_status(sq_pool* pool, int32_t* device_flag) {
   if (device_flag) *device_flag = f;
   if (f & SQ_FLAG_TIMEOUT) return SQ_ERR_TIMEOUT;
   return f ? SQ_ERR_DEVICE_FLAG : SQ_OK;
+}
+
+sq_status sq_debug_set_wait(sq_pool* pool, uint64_t wait_limit_ns, uint32_t extra_expected_bytes) {
+  if (!pool || extra_expected_bytes > 4096u) return SQ_ERR_INVALID_ARG;
+  pool->wait_ns = wait_limit_ns ? wait_limit_ns : 1000000000ull;
+  pool->extra_tx = extra_expected_bytes;
+  return SQ_OK;
 }
 
 const char* sq_status_string(sq_status status) {

@@ -56,9 +56,13 @@ struct StepArgs {
   int64_t side_slot_bytes, side_head_bytes;
   int32_t window, n_outliers;
   int32_t n_tok;  // tokens of a chunk (sq_decode_chunk)
-  const float* rho;  // null, or [H][d_k] row impact / the head's largest (sq_pool_set_row_impact)
+  const float* omega;  // null, or [H][d_k] column-pass weights of the impact-weighted fit
+                       // (sq_pool_set_row_impact)
   int32_t update_only;  // with s_new: write the updated fp32 state and stop (no refit, no
                         // requantization); a skipped item gets a NaN in its s_new block
+  uint64_t wait_ns;     // limit of every wait on a bulk copy (global-timer nanoseconds)
+  uint32_t extra_tx;    // test hook: bytes the decode kernel's stage barrier expects beyond
+                        // what its copies bring (0 in normal use; > 0 makes the wait run out)
 };
 
 struct QuantArgs {
@@ -68,7 +72,7 @@ struct QuantArgs {
   const int32_t* slot_idx;
   int32_t n;
   const float* S;  // quantize: input; dequantize: output (cast away const)
-  const float* rho;  // null, or [H][d_k] row impact weights (as StepArgs::rho)
+  const float* omega;  // null, or [H][d_k] column-pass weights (as StepArgs::omega)
   float* S_out;
   const HeadDesc* heads;
   const uint32_t* rows;

@@ -9,34 +9,25 @@
 // exits.
 #include <cuda_runtime.h>
 
-#include <mutex>
-
 #include "sq.h"
 #include "sq_internal.h"
 
 namespace {
 
 constexpr size_t kStagingBytes = size_t(32) << 20;  // 32 MiB: 512 request-heads at d = 128
-constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_staging[kStagingBytes];
 
-std::mutex g_mu;
-float* g_staging_addr[kMaxDevices] = {};
-
-// Device address of g_staging on the current device; looked up on the first call per device.
-// (In host code `g_staging` names a host-side stand-in, not device memory.)
+// Device address of g_staging on the current device, looked up on every call (the lookup
+// allocates nothing and costs little; a cached address would go stale if the device's context
+// were torn down and created again). In host code `g_staging` names a host-side stand-in, not
+// device memory, so it is never passed to a kernel itself. The first lookup on a device may
+// load the library's module there, which is why the first call should come before any stream
+// capture.
 sq_status staging_on_current_device(float** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return SQ_ERR_CUDA;
-  if (dev < 0 || dev >= kMaxDevices) return SQ_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_staging_addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_staging) != cudaSuccess || !p) return SQ_ERR_CUDA;
-    g_staging_addr[dev] = static_cast<float*>(p);
-  }
-  *out = g_staging_addr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_staging) != cudaSuccess || !p) return SQ_ERR_CUDA;
+  *out = static_cast<float*>(p);
   return SQ_OK;
 }
 

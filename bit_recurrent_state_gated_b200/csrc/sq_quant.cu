@@ -50,8 +50,8 @@ __global__ void __launch_bounds__(kThreads) k_quantize(const QuantArgs a) {
     return;
   }
   uint8_t* dst = a.pool + (size_t)slot * a.slot_bytes + hd.off;
-  const float* rho = a.rho ? a.rho + (size_t)h * dk : nullptr;
-  const bool ok = quantize_tile(S, dst, hd, rows, rho, a.n_outliers, a.fit_iters, warp, lane, dk,
+  const float* omega = a.omega ? a.omega + (size_t)h * dk : nullptr;
+  const bool ok = quantize_tile(S, dst, hd, rows, omega, a.n_outliers, a.fit_iters, warp, lane, dk,
                                 dv, sm);
   if (!ok && tid == 0) atomicOr(a.flag, SQ_FLAG_RANGE_BIT);
   if (a.side && tid == 0)  // close this head's window

@@ -43,12 +43,13 @@ __device__ __forceinline__ int q_of_width(int b) { return b == 16 ? 0 : (1 << (b
 // w_i = fl(1 / fl(r_i Q_i)); c_j = max(max_i fl(|S_ij| w_i), 2^-14). Rows with Q = 0 (fp16
 // pivot rows) get w = 0 and drop out of the column maxima; zeroed elements (outliers, idle
 // lanes) contribute nothing. On return rowR[i] = r_i and col[COL_X][j] = c_j.
-// Row impact (rho, per row of the head, in (0, 1], or null): a row's scale widens to
-// min(fl(q_i / rho_i), 65504) when that is larger than q_i = fl(m_i / Q_i), so its w_i shrinks
-// and the column scales follow the high-impact rows.
+// Row weights (omega, per row of the head, in (0, 1], or null; impact-weighted pools): a row
+// weighted below 1 counts in the column passes with w_i = fl(omega_i fl(1 / fl(r_i Q_i))), so
+// the column scales follow the high-impact rows, and after the last alternation it is fit once
+// more against the final column scales, r_i = max(r_i, fl(max_j fl(|S_ij| fl(1/c_j)) / Q_i)).
 __device__ __forceinline__ void fit_scales(const float (&S)[kRows][4], int fit_iters, int warp,
                                            int lane, int dk, int dv, const uint32_t* rows,
-                                           const float* rho, float* rowW, float* rowR,
+                                           const float* omega, float* rowW, float* rowR,
                                            float* rowtmp, float* red, float* col) {
   float inv_c[4] = {1.f, 1.f, 1.f, 1.f};
   float* tmp = rowtmp + warp * kRows;
@@ -78,8 +79,8 @@ __device__ __forceinline__ void fit_scales(const float (&S)[kRows][4], int fit_i
         if (Q > 0) {
           const float q = __fdiv_rn(tmp[lane], (float)Q);
           r = fmaxf(q, kScaleFloor);
-          if (rho) r = fmaxf(r, fminf(__fdiv_rn(q, rho[i]), 65504.f));
           w = __frcp_rn(__fmul_rn(r, (float)Q));
+          if (omega && omega[i] < 1.f) w = __fmul_rn(omega[i], w);
         }
         rowR[i] = r;
         rowW[i] = w;
@@ -115,13 +116,34 @@ __device__ __forceinline__ void fit_scales(const float (&S)[kRows][4], int fit_i
       col[COL_INV * kMaxD + t] = 1.f;
     }
     __syncthreads();
-    if (it + 1 < fit_iters) {
+    if (it + 1 < fit_iters || omega) {
       const float4 iv = *reinterpret_cast<const float4*>(col + COL_INV * kMaxD + 4 * lane);
       inv_c[0] = iv.x;
       inv_c[1] = iv.y;
       inv_c[2] = iv.z;
       inv_c[3] = iv.w;
     }
+  }
+  if (omega) {  // rows weighted below 1: fit once more against the final column scales
+    float rm[kRows];
+#pragma unroll
+    for (int s = 0; s < kRows; ++s)
+      rm[s] = warp_max_nonneg(fmaxf(fmaxf(fabsf(S[s][0]) * inv_c[0], fabsf(S[s][1]) * inv_c[1]),
+                                    fmaxf(fabsf(S[s][2]) * inv_c[2], fabsf(S[s][3]) * inv_c[3])));
+    if (lane == 0) {
+#pragma unroll
+      for (int s = 0; s < kRows; s += 4)
+        *reinterpret_cast<float4*>(tmp + s) = make_float4(rm[s], rm[s + 1], rm[s + 2], rm[s + 3]);
+    }
+    __syncwarp();
+    if (lane < kRows) {
+      const int i = warp * kRows + lane;
+      if (i < dk && omega[i] < 1.f) {
+        const int Q = q_of_width(row_width(rows[i]));
+        if (Q > 0) rowR[i] = fmaxf(rowR[i], __fdiv_rn(tmp[lane], (float)Q));
+      }
+    }
+    __syncthreads();
   }
 }
 
@@ -484,7 +506,7 @@ __device__ __forceinline__ void select_top_fast(const float (&S)[kRows][4], int 
 // stored) on an fp16 range overflow. Contains __syncthreads; sm.misc[0] must be 0 on entry.
 __device__ __forceinline__ bool quantize_tile(float (&S)[kRows][4], uint8_t* dst,
                                               const HeadDesc& hd, const uint32_t* rows,
-                                              const float* rho, int n_out, int fit_iters,
+                                              const float* omega, int n_out, int fit_iters,
                                               int warp, int lane, int dk, int dv, TileSmem& sm) {
   if (hd.pivot_head) return store_pivot_head(S, dst, warp, lane, dk, dv, &sm.misc[0]);
   if (n_out > 0) {
@@ -498,7 +520,7 @@ __device__ __forceinline__ bool quantize_tile(float (&S)[kRows][4], uint8_t* dst
     if ((int)threadIdx.x < n_out && __hisinf(__float2half_rn(sm.oval[threadIdx.x])))
       atomicOr(&sm.misc[0], 1);
   }
-  fit_scales(S, fit_iters, warp, lane, dk, dv, rows, rho, sm.rowW, sm.rowR, sm.rowtmp, sm.red,
+  fit_scales(S, fit_iters, warp, lane, dk, dv, rows, omega, sm.rowW, sm.rowR, sm.rowtmp, sm.red,
              sm.col);
   const bool ok = requant_store_any(mode_of(hd), S, dst, rows, warp, lane, dk, dv, sm.rowR,
                                     sm.rowIR, sm.col, &sm.misc[0]);

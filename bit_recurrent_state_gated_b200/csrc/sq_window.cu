@@ -94,7 +94,7 @@ __device__ __forceinline__ void flush_tile(const StepArgs& a, TileSmem& ts, cons
                                            const float* terms, int nterms, const float* g,
                                            bool add_new, const float* kk, const float* bcol,
                                            uint8_t* dst, const HeadDesc& hd,
-                                           const uint32_t* rows, const float* rho,
+                                           const uint32_t* rows, const float* omega,
                                            int32_t* count) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, dk = a.dk, dv = a.dv;
   float S[kRows][4];
@@ -130,7 +130,7 @@ __device__ __forceinline__ void flush_tile(const StepArgs& a, TileSmem& ts, cons
   }
   if (tid == 0) ts.misc[0] = 0;
   __syncthreads();
-  const bool ok = quantize_tile(S, dst, hd, rows, rho, a.n_outliers, a.fit_iters, warp, lane, dk,
+  const bool ok = quantize_tile(S, dst, hd, rows, omega, a.n_outliers, a.fit_iters, warp, lane, dk,
                                 dv, ts);
   if (!ok && tid == 0) atomicOr(a.flag, SQ_FLAG_RANGE_BIT);
   if (tid == 0) *count = 0;
@@ -161,7 +161,7 @@ __global__ void __launch_bounds__(kThreads) k_window_flush(const StepArgs a) {
   copy16(sm.g, side + 16, dk * 4, a.flag);
   __syncthreads();
   flush_tile(a, sm.t, blk, terms, cnt, sm.g, false, nullptr, nullptr, dst, hd, rows,
-             a.rho ? a.rho + (size_t)h * dk : nullptr, count);
+             a.omega ? a.omega + (size_t)h * dk : nullptr, count);
   (void)tid;
 }
 

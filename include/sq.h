@@ -185,9 +185,10 @@ SQ_API sq_status sq_decode_step_split(sq_pool* pool, const int32_t* slot_idx, in
  * point allocates nothing. The pages have no counterpart: it only serves such callers.
  *   batch * n_heads * d_k * d_v * 4 bytes must fit in 32 MiB (512 request-heads at
  *   d = 128); larger batches return SQ_ERR_INVALID_ARG.
- * Both halves (update, then refit + requantize) run on `stream`. The first call on a device
- * (with that device current) looks up the array's device address; make that first call
- * before any stream capture. All calls in the process share the one array and it keeps the
+ * Both halves (update, then refit + requantize) run on `stream`. Every call looks up the
+ * array's device address on the current device (no address is cached, so a context torn down
+ * and created again is harmless); the first call on a device may load the library's module
+ * there, so make that first call before any stream capture. All calls in the process share the one array and it keeps the
  * last call's contents (nothing in it needs to start at zero: each call writes every tile it
  * reads back); calls that can run at the same time on the GPU (different streams, different
  * pools) race on it and must be ordered by the caller. Other arguments and errors as
@@ -226,13 +227,14 @@ SQ_API sq_status sq_window_flush(sq_pool* pool, const int32_t* slot_idx, int32_t
  * penalizes reconstruction error more in high-impact rows; the impact scores are fixed
  * offline, [SQ-E] row-impact score paragraph). impact (host) fp32 [n_heads][d_k], every entry
  * > 0 and finite, or NULL to remove the weighting. Reading taken (the pages print no
- * formula): rho_i = impact_i / (largest impact of the head) in fp64, rounded to fp32; in
- * every refit of the pool (decode step, chunk, window end, quantize, flush) the row scale
- * becomes r_i = max(q_i, min(q_i / rho_i, 65504), 2^-14) with q_i = m_i / Q_i (m_i the row's
- * max-abs over the current column scales), so low-impact rows take wider steps and the column
- * scales follow the high-impact rows; no code leaves [-Q, Q]. Synchronizes the device;
- * allocates a small device table on first use. SQ_ERR_INVALID_ARG for a bad entry (the
- * previous weighting stays). */
+ * formula): row i of head h counts in the column passes of every refit of the pool (decode
+ * step, chunk, window end, quantize, flush) with the weight omega_i = min(1, sqrt(impact_i /
+ * mean impact of head h)) (double precision, rounded to fp32), i.e. w_i = omega_i / (r_i Q_i),
+ * so the column scales follow the high-impact rows; after the last alternation every row with
+ * omega_i < 1 widens its scale to fit the final column scales, so no code leaves [-Q, Q].
+ * Each row scale otherwise follows the row's own size. Equal impacts give the plain fit.
+ * Synchronizes the device; allocates a small device table on first use. SQ_ERR_INVALID_ARG for
+ * a bad entry (the previous weighting stays). */
 SQ_API sq_status sq_pool_set_row_impact(sq_pool* pool, const float* impact);
 
 /* Synchronize the device, read and clear the status word (*device_flag, may be NULL).
@@ -270,6 +272,20 @@ SQ_API sq_status sq_debug_decode_step_fp32(sq_pool* pool, const int32_t* slot_id
                                     const void* q, const void* k, const void* v,
                                     const float* alpha, const float* beta, float* out,
                                     float* s_new, void* stream);
+
+/*
+ * Test hook for the bounded waits (the pages have no counterpart: it exists so that the
+ * timeout path can be exercised without faulting anything). Every later sq_decode_step and
+ * sq_debug_decode_step_fp32 on this pool (window == 1) gives up a wait on a bulk copy after
+ * wait_limit_ns nanoseconds of the GPU's global timer (0 restores the default, 1 s), and, with
+ * extra_expected_bytes > 0 (at most 4096), has each copy's barrier expect that many bytes more
+ * than the copies bring, so that every wait runs out. A kernel whose wait runs out sets
+ * SQ_FLAG_TIMEOUT (sq_pool_status then returns SQ_ERR_TIMEOUT), lets its own copies land, frees
+ * its tensor memory and returns; the items it did not reach keep their slot bytes and their
+ * output rows are not written. Host only; nothing is enqueued. Call with 0, 0 to restore normal
+ * operation. SQ_ERR_INVALID_ARG for a NULL pool or more than 4096 extra bytes. */
+SQ_API sq_status sq_debug_set_wait(sq_pool* pool, uint64_t wait_limit_ns,
+                                   uint32_t extra_expected_bytes);
 
 #ifdef __cplusplus
 }

@@ -17,7 +17,7 @@ def lib():
 
 def test_exports_every_declared_symbol(lib):
     names = sq.exported_names()
-    assert len(names) == 16, names  # the calls include/sq.h declares
+    assert len(names) == 17, names  # the calls include/sq.h declares
     for n in names:
         assert hasattr(lib, n), n
 
@@ -89,3 +89,7 @@ def test_calls_on_null_pool_rejected(lib):
     with pytest.raises(sq.SqError):
         sq.sq_decode_step_split_static(0, 16, 1, 16, 16, 16, 16, 16, 16, 0)
     sq.sq_state_pool_destroy(0)
+
+
+def test_set_wait_rejects_a_null_pool(lib):
+    assert lib.sq_debug_set_wait(None, 1000, 0) == sq.SQ_ERR_INVALID_ARG

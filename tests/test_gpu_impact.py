@@ -1,7 +1,8 @@
 """GPU parity of the row-impact weighted fit (sq_pool_set_row_impact) against the CPU oracle.
 
-The weighting changes only the row scales of every refit (r_i = max(q_i, min(q_i / rho_i,
-65504), 2^-14)); the cold-start quantization must stay bit-exact with the oracle's, and the
+The weighting changes the column passes of every refit (row i counts with the weight
+min(1, sqrt(impact_i / mean impact)), and rows weighted below 1 are fit once more against the
+final column scales); the cold-start quantization must stay bit-exact with the oracle's, and the
 decode step, the chunk step and the window end must follow the oracle within the lockstep
 bounds. Impacts are seeded log-uniform scores over two decades.
 """
