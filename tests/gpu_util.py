@@ -97,22 +97,76 @@ def close(got, ref, what: str):
 
 def compare_codes(wl, bits, gpu_slots: np.ndarray, orc_slots: np.ndarray, what: str):
     """Codes equal on >= 99.99 % of quantized elements and within 1 LSB elsewhere; the
-    dequantized states within tolerance wherever codes match (fp16 entries always)."""
-    dg = packed.decode(gpu_slots, wl.unit, bits, wl.n_heads, wl.d_k, wl.d_v, wl.n_outliers)
-    do = packed.decode(orc_slots, wl.unit, bits, wl.n_heads, wl.d_k, wl.d_v, wl.n_outliers)
-    quant = ~np.broadcast_to(dg["pivot"][None, :, :, None], dg["codes"].shape)
-    if wl.n_outliers:
-        quant = quant & (dg["f16"] == 0) & (do["f16"] == 0)
-    diff = np.abs(dg["codes"] - do["codes"])[quant]
-    n_mis = int((diff != 0).sum())
-    frac = n_mis / max(diff.size, 1)
-    assert diff.size == 0 or diff.max() <= 1, f"{what}: code differs by {diff.max()} LSB"
-    if diff.size >= 100_000:  # on small samples one flip exceeds the fraction; callers sum up
-        assert frac <= 1e-4, f"{what}: {n_mis} of {diff.size} codes differ ({frac:.2e})"
-    Dg, Do = packed.dequant(dg), packed.dequant(do)
-    same = (dg["codes"] == do["codes"]) | ~quant
-    close(Dg[same], Do[same], what + " dequantized state")
-    return n_mis, diff.size
+    dequantized states within tolerance wherever codes match (fp16 entries always). Head
+    blocks whose bytes are identical on both sides agree trivially; only the others are
+    decoded and compared element by element."""
+    H, dk, dv, K = wl.n_heads, wl.d_k, wl.d_v, wl.n_outliers
+    ranges = packed.head_ranges(wl.unit, bits, H, dk, dv, K)
+    n_mis = total = 0
+    max_diff = 0
+    for h, (a, b) in enumerate(ranges):
+        bh = packed.head_bits(wl.unit, bits, h, dk)
+        if wl.unit == W.UNIT_HEAD:
+            n_quant = 0 if bh[0] == 16 else dk * dv - K
+        else:
+            n_quant = int((bh != 16).sum()) * dv - K
+        differ = np.nonzero((gpu_slots[:, a:b] != orc_slots[:, a:b]).any(axis=1))[0]
+        total += n_quant * gpu_slots.shape[0]
+        if differ.size == 0:
+            continue
+        dg = packed.decode(gpu_slots[differ, a:b], wl.unit, bh, 1, dk, dv, K)
+        do = packed.decode(orc_slots[differ, a:b], wl.unit, bh, 1, dk, dv, K)
+        quant = ~np.broadcast_to(dg["pivot"][None, :, :, None], dg["codes"].shape)
+        if K:
+            quant = quant & (dg["f16"] == 0) & (do["f16"] == 0)
+        diff = np.abs(dg["codes"] - do["codes"])[quant]
+        n_mis += int((diff != 0).sum())
+        if diff.size:
+            max_diff = max(max_diff, int(diff.max()))
+        Dg, Do = packed.dequant(dg), packed.dequant(do)
+        same = (dg["codes"] == do["codes"]) | ~quant
+        close(Dg[same], Do[same], f"{what} head {h} dequantized state")
+    assert max_diff <= 1, f"{what}: code differs by {max_diff} LSB"
+    frac = n_mis / max(total, 1)
+    if total >= 100_000:  # on small samples one flip exceeds the fraction; callers sum up
+        assert frac <= 1e-4, f"{what}: {n_mis} of {total} codes differ ({frac:.2e})"
+    return n_mis, total
+
+
+def code_agreement(wl, bits, slots_a: np.ndarray, slots_b: np.ndarray):
+    """Element statistics of two packed copies of the same requests: (quantized elements,
+    of them with equal codes, of those whose dequantized values are within tolerance, the
+    largest dequantized difference among them). Identical head blocks count as agreeing."""
+    H, dk, dv, K = wl.n_heads, wl.d_k, wl.d_v, wl.n_outliers
+    n_quant = n_agree = n_ok = 0
+    max_err = 0.0
+    for h, (a, b) in enumerate(packed.head_ranges(wl.unit, bits, H, dk, dv, K)):
+        bh = packed.head_bits(wl.unit, bits, h, dk)
+        if wl.unit == W.UNIT_HEAD:
+            per = 0 if bh[0] == 16 else dk * dv - K
+        else:
+            per = int((bh != 16).sum()) * dv - K
+        differ = (slots_a[:, a:b] != slots_b[:, a:b]).any(axis=1)
+        same_n = int((~differ).sum()) * per
+        n_quant, n_agree, n_ok = n_quant + same_n, n_agree + same_n, n_ok + same_n
+        idx = np.nonzero(differ)[0]
+        if idx.size == 0 or per == 0:
+            n_quant += idx.size * per
+            continue
+        da = packed.decode(slots_a[idx, a:b], wl.unit, bh, 1, dk, dv, K)
+        db = packed.decode(slots_b[idx, a:b], wl.unit, bh, 1, dk, dv, K)
+        quant = ~np.broadcast_to(da["pivot"][None, :, :, None], da["codes"].shape)
+        if K:
+            quant = quant & (da["f16"] == 0) & (db["f16"] == 0)
+        agree = (da["codes"] == db["codes"]) & quant
+        Da, Db = packed.dequant(da).astype(np.float64), packed.dequant(db)
+        err = np.abs(Da - Db)[agree]
+        n_quant += int(quant.sum())
+        n_agree += int(agree.sum())
+        n_ok += int((err <= ATOL + RTOL * np.abs(np.asarray(Db, np.float64)[agree])).sum())
+        if err.size:
+            max_err = max(max_err, float(err.max()))
+    return n_quant, n_agree, n_ok, max_err
 
 
 def lockstep(case: GpuCase, t: int, sample=None, want_state=True, x=None):

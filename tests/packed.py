@@ -103,6 +103,28 @@ def decode(slots: np.ndarray, unit: int, bits, H: int, dk: int, dv: int, n_outli
                 widths=W)
 
 
+def head_ranges(unit: int, bits, H: int, dk: int, dv: int, n_outliers: int = 0):
+    """[(start, end)] byte range of each head block within a slot (end includes the padding)."""
+    W, _, head_off, _ = _plan(unit, bits, H, dk, dv, n_outliers)
+    ends = list(head_off[1:]) + [None]
+    out = []
+    for h in range(H):
+        if ends[h] is None:
+            if unit == 0 and W[h, 0] == 16:
+                size = 2 * dk * dv
+            else:
+                size = 2 * (dk + dv) + sum(dv * int(b) // 8 for b in W[h]) + 4 * n_outliers
+            ends[h] = head_off[h] + (size + 15) // 16 * 16
+        out.append((int(head_off[h]), int(ends[h])))
+    return out
+
+
+def head_bits(unit: int, bits, h: int, dk: int) -> np.ndarray:
+    """The bit map of head h alone (a one-head layout)."""
+    b = np.asarray(bits, np.uint8)
+    return b[h:h + 1] if unit == 0 else b[h * dk:(h + 1) * dk]
+
+
 def dequant(d) -> np.ndarray:
     """fp32 state from a decoded pool: code * r16 * c16, fp16 values where stored."""
     D = (d["codes"] * d["r16"][..., None] * d["c16"][:, :, None, :]).astype(np.float32)
