@@ -53,3 +53,5 @@ def test_chunk_and_window_amortize_the_state():
     reads = sum(t * 4 * 2 * D + (4 * D if t else 0) for t in range(16))
     writes = 15 * (4 * 2 * D + 4 * D + 4)
     assert ab["side"] == H * (reads + writes) / 16
+    # the side state is this implementation's representation: reported apart, not in the total
+    assert ab["total"] == 541_696 + 541_696 / 16 + IO_BF16_SCALAR == 616_772
