@@ -35,6 +35,7 @@ struct sq_pool {
   // bounded waits of the decode kernel (sq_debug_set_wait)
   uint64_t wait_ns = 1000000000ull;
   uint32_t extra_tx = 0;
+  int32_t full_fit = 0;  // sq_debug_set_full_fit
 };
 
 namespace sq {
@@ -193,6 +194,7 @@ sq::StepArgs step_args(sq_pool* p, const int32_t* slot_idx, int32_t batch, const
   a.omega = p->has_omega ? p->d_omega : nullptr;
   a.wait_ns = p->wait_ns;
   a.extra_tx = p->extra_tx;
+  a.full_fit = p->full_fit;
   return a;
 }
 
@@ -486,6 +488,12 @@ sq_status sq_debug_set_wait(sq_pool* pool, uint64_t wait_limit_ns, uint32_t extr
   if (!pool || extra_expected_bytes > 4096u) return SQ_ERR_INVALID_ARG;
   pool->wait_ns = wait_limit_ns ? wait_limit_ns : 1000000000ull;
   pool->extra_tx = extra_expected_bytes;
+  return SQ_OK;
+}
+
+sq_status sq_debug_set_full_fit(sq_pool* pool, int32_t full_fit) {
+  if (!pool || (full_fit != 0 && full_fit != 1)) return SQ_ERR_INVALID_ARG;
+  pool->full_fit = full_fit;
   return SQ_OK;
 }
 

@@ -48,13 +48,13 @@ __device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
 }
 
 // Pass A of a later token: Sbar^T y and Sbar^T z from the codes held in tensor memory.
-template <bool FULL>
-__device__ __forceinline__ void pass_a_tmem(const Ctx<FULL>& c) {
+template <class C>
+__device__ __forceinline__ void pass_a_tmem(const C& c) {
   const float4* gkq = sp<float4>(S_GKQ) + c.row0() / 2;
   float2 U[4], P[4];
 #pragma unroll
   for (int e = 0; e < 4; ++e) U[e] = P[e] = f2(0.f, 0.f);
-  sweep(c.tm, c.nch(), [&](int ch, float2 (&v)[8]) {
+  sweep(c, [&](int ch, float2 (&v)[8]) {
 #pragma unroll
     for (int pr = 0; pr < 2; ++pr) {
       const float4 g = gkq[2 * ch + pr];
@@ -100,7 +100,7 @@ __device__ __forceinline__ void rebase_tile(const Ctx<FULL>& c, const float* ter
   const float4* ak = sp<float4>(S_AK) + c.row0() / 2;
   const float2* gnp = reinterpret_cast<const float2*>(sp<float>(W_GNP) + c.row0());
   const uint4* rd4 = reinterpret_cast<const uint4*>(sp<uint32_t>(S_RD) + c.row0());
-  sweep(c.tm, c.nch(), [&](int ch, float2 (&v)[8]) {
+  sweep(c, [&](int ch, float2 (&v)[8]) {
     const uint4 d = rd4[ch];
     float2 acc[8];
 #pragma unroll

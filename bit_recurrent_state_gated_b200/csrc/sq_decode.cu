@@ -49,7 +49,7 @@ template <int GATE, int IO, bool WS, bool FULL, bool ROWS>
 __global__ void __launch_bounds__(kT, kMaxCtasPerSm) k_decode(const StepArgs a) {
   const DPlan P(a.dk, a.dv, IO, GATE, ROWS, a.stage_bytes, a.H);
   uint64_t* bar = sp<uint64_t>(S_BAR);
-  Ctx<FULL> c;
+  Ctx<FULL, !ROWS> c;
   c.tid = threadIdx.x;
   c.warp = c.tid >> 5;
   c.lane = c.tid & 31;
@@ -208,7 +208,8 @@ __global__ void __launch_bounds__(kT, kMaxCtasPerSm) k_decode(const StepArgs a) 
         akp[0] = A;
         akp[2] = ki;
         const bool okA = A >= 0x1p-60f && A <= 0x1p60f;  // k / A representable to full precision
-        sp<float>(S_KT)[p] = okA ? __fdiv_rn(ki, A) : 0.f;
+        // k / A within 2 ulps (the tile's own factor, not a quantizer decision)
+        sp<float>(S_KT)[p] = okA ? ki * rcp_approx(A) : 0.f;
         bad_a = !okA;
         kqp = ki * qi;
       }
@@ -320,15 +321,26 @@ __global__ void __launch_bounds__(kT, kMaxCtasPerSm) k_decode(const StepArgs a) 
     __syncthreads();  // barrier 2
     float4 cm = max4(sp<float>(S_REDC), c.lane);
     for (int f = 1; f < a.fit_iters; ++f) {
-      row_pass(c, make_float4(__frcp_rn(cm.x), __frcp_rn(cm.y), __frcp_rn(cm.z), __frcp_rn(cm.w)));
+      // the last column pass may be skipped (see column_slack); not with row weights, whose
+      // closing refit needs the exact fp32 column scales
+      const bool maybe_skip = f + 1 == a.fit_iters && !a.omega && !a.full_fit;
+      if (maybe_skip) column_slack(c.warp, c.lane, cm, c.act());
+      const float w_old = sp<float>(S_W)[c.row0() + c.lane];
+      row_pass(c, make_float4(rcp_rn(cm.x), rcp_rn(cm.y), rcp_rn(cm.z), rcp_rn(cm.w)));
       r = row_scales(c, false, omega);
+      if (maybe_skip) {
+        multiplier_change(c.warp, c.lane, w_old, sp<float>(S_W)[c.row0() + c.lane]);
+        __syncthreads();  // barrier 3 (fit_iters = 2): slack and changes of every warp
+        const float4 d4 = *sp<float4>(S_FIT);
+        if (fmaxf(fmaxf(d4.x, d4.y), fmaxf(d4.z, d4.w)) <= sp<float>(S_FIT)[4]) break;
+      }
       float* red = sp<float>(S_REDC) + (f & 1) * kW * kMaxD;
       col_pass(c, red);
-      __syncthreads();  // barrier 3 (fit_iters = 2)
+      __syncthreads();  // barrier 3 (or 4 after a failed skip test)
       cm = max4(red, c.lane);
     }
     if (a.omega) {  // rows weighted below 1: fit once more against the final column scales
-      row_pass(c, make_float4(__frcp_rn(cm.x), __frcp_rn(cm.y), __frcp_rn(cm.z), __frcp_rn(cm.w)));
+      row_pass(c, make_float4(rcp_rn(cm.x), rcp_rn(cm.y), rcp_rn(cm.z), rcp_rn(cm.w)));
       r = row_refit(c, r, omega);
       __syncthreads();  // every warp sees the range flags the refit may have set
     }

@@ -94,8 +94,8 @@ __device__ __forceinline__ void chunk_add(float2 (&v)[8], int r, int e, float ad
 // One element of the tensor-memory tile, by processing row p and column j: its owner warp loads
 // the chunk, the owner lane changes the element (x += add, or x = add), the warp stores it.
 // Returns the element's new value to the owner lane (0 elsewhere).
-template <bool FULL>
-__device__ __forceinline__ float tile_patch(const Ctx<FULL>& c, int p, int j, float add, bool set) {
+template <class C>
+__device__ __forceinline__ float tile_patch(const C& c, int p, int j, float add, bool set) {
   if (p / kRW != c.warp) return 0.f;  // warp-uniform
   const int ch = (p % kRW) / 4;
   uint32_t r[16];
@@ -137,7 +137,7 @@ __device__ __forceinline__ void window_fold(const Ctx<FULL>& c, const StepArgs& 
   // ---- materialize S = g (x A c + sum_s k_hat_s b_s^T) + k b^T in tensor memory; the thread's
   // largest |S| over the rows eligible for compensation entries ----
   float tmaxf = 0.f;
-  sweep(c.tm, c.nch(), [&](int ch, float2 (&v)[8]) {
+  sweep(c, [&](int ch, float2 (&v)[8]) {
     const uint4 d = rd4[ch];
     const int orow[4] = {rd_row(d.x), rd_row(d.y), rd_row(d.z), rd_row(d.w)};
     float2 acc[8];
@@ -229,7 +229,7 @@ __device__ __forceinline__ void window_fold(const Ctx<FULL>& c, const StepArgs& 
     }
     __syncthreads();
     const uint32_t thr = (uint32_t)misc[1];
-    sweep(c.tm, c.nch(), [&](int ch, float2 (&v)[8]) {
+    sweep(c, [&](int ch, float2 (&v)[8]) {
       float cmx = 0.f;  // the chunk's largest |S| (all rows) bounds its candidates
 #pragma unroll
       for (int e = 0; e < 8; ++e) cmx = max3abs(cmx, v[e].x, v[e].y);
@@ -305,7 +305,7 @@ __device__ __forceinline__ void window_fold(const Ctx<FULL>& c, const StepArgs& 
         unsigned long long best = 0;
         int bp = 0;
         float bvx = 0.f;
-        sweep(c.tm, c.nch(), [&](int ch, float2 (&v)[8]) {
+        sweep(c, [&](int ch, float2 (&v)[8]) {
           const uint4 d = rd4[ch];
           const uint32_t ds[4] = {d.x, d.y, d.z, d.w};
 #pragma unroll
@@ -373,7 +373,7 @@ __device__ __forceinline__ void window_fold(const Ctx<FULL>& c, const StepArgs& 
   // ---- refit and requantize (pivot heads: round to fp16) ----
   if (pivot_head) {
     bool of = false;
-    sweep(c.tm, c.nch(), [&](int ch, float2 (&v)[8]) {
+    sweep(c, [&](int ch, float2 (&v)[8]) {
       float m = 0.f;
 #pragma unroll
       for (int e = 0; e < 8; ++e) m = max3abs(m, v[e].x, v[e].y);
@@ -392,7 +392,7 @@ __device__ __forceinline__ void window_fold(const Ctx<FULL>& c, const StepArgs& 
   {  // row maxima (fp16 rows: range check)
     float4* rtab = reinterpret_cast<float4*>(sp<float>(S_RT) + c.row0());
     bool of = false;
-    sweep(c.tm, c.nch(), [&](int ch, float2 (&v)[8]) {
+    sweep(c, [&](int ch, float2 (&v)[8]) {
       float rm[4];
 #pragma unroll
       for (int pr = 0; pr < 2; ++pr) {
@@ -416,7 +416,7 @@ __device__ __forceinline__ void window_fold(const Ctx<FULL>& c, const StepArgs& 
   __syncthreads();
   float4 cm = max4(sp<float>(S_REDC), lane);
   for (int f = 1; f < a.fit_iters; ++f) {
-    row_pass(c, make_float4(__frcp_rn(cm.x), __frcp_rn(cm.y), __frcp_rn(cm.z), __frcp_rn(cm.w)));
+    row_pass(c, make_float4(rcp_rn(cm.x), rcp_rn(cm.y), rcp_rn(cm.z), rcp_rn(cm.w)));
     r = row_scales(c, false, omega);
     float* red = sp<float>(S_REDC) + (f & 1) * kW * kMaxD;
     col_pass(c, red);
@@ -424,7 +424,7 @@ __device__ __forceinline__ void window_fold(const Ctx<FULL>& c, const StepArgs& 
     cm = max4(red, lane);
   }
   if (a.omega) {  // rows weighted below 1: fit once more against the final column scales
-    row_pass(c, make_float4(__frcp_rn(cm.x), __frcp_rn(cm.y), __frcp_rn(cm.z), __frcp_rn(cm.w)));
+    row_pass(c, make_float4(rcp_rn(cm.x), rcp_rn(cm.y), rcp_rn(cm.z), rcp_rn(cm.w)));
     r = row_refit(c, r, omega);
     __syncthreads();  // every warp sees the range flags the refit may have set
   }

@@ -63,6 +63,7 @@ struct StepArgs {
   uint64_t wait_ns;     // limit of every wait on a bulk copy (global-timer nanoseconds)
   uint32_t extra_tx;    // test hook: bytes the decode kernel's stage barrier expects beyond
                         // what its copies bring (0 in normal use; > 0 makes the wait run out)
+  int32_t full_fit;     // test hook: 1 = never skip the last column pass of the fit
 };
 
 struct QuantArgs {

@@ -62,7 +62,9 @@ constexpr uint32_t S_REDP = S_REDU + 2048;    // [4 warps][128] partial P
 constexpr uint32_t S_REDC = S_REDP + 2048;    // [2][4 warps][128] partial column maxima
 constexpr uint32_t S_KT = S_REDC + 4096;      // float per row: k_i / A_i
 constexpr uint32_t S_TR = S_KT + 512;         // float per row: t_i, the tile holds M_ij / t_i
-constexpr uint32_t S_STAGE = S_TR + 512;      // staging buffer, then the head table
+constexpr uint32_t S_FIT = S_TR + 512;        // [4] per-warp change of the column multipliers,
+                                              // [4] slack of the column scales (last column pass)
+constexpr uint32_t S_STAGE = S_FIT + 32;      // staging buffer, then the head table
 static_assert(S_STAGE % 16 == 0 && S_GKQ % 16 == 0 && S_REDU % 16 == 0, "16-byte aligned");
 
 // Row descriptor, processing order: original row << 24 | byte offset in the block << 8 | width.
@@ -138,7 +140,7 @@ __device__ __forceinline__ void tm_take(uint32_t (&r)[16], float2 (&v)[8]) {
 // Run body(ch, v) over chunks 0..nch-1 (nch even) of the thread's tile, each chunk's load in
 // flight while the previous chunk is processed.
 template <class F>
-__device__ __forceinline__ void sweep(uint32_t tm, int nch, F&& body) {
+__device__ __forceinline__ void sweep_ahead(uint32_t tm, int nch, F&& body) {
   uint32_t ra[16], rb[16];
   if (nch <= 0) return;
   tm_issue(tm, ra);
@@ -153,6 +155,28 @@ __device__ __forceinline__ void sweep(uint32_t tm, int nch, F&& body) {
     if (ch + 2 < nch) tm_issue(tm + 16u * (ch + 2), ra);
     body(ch + 1, w);
   }
+}
+
+// The same, one chunk at a time (a smaller loop: the key-row kernels, whose bodies dispatch
+// on row widths, run faster this way).
+template <class F>
+__device__ __forceinline__ void sweep_each(uint32_t tm, int nch, F&& body) {
+#pragma unroll 1
+  for (int ch = 0; ch < nch; ++ch) {
+    uint32_t r[16];
+    float2 v[8];
+    tm_issue(tm + 16u * ch, r);
+    tm_take(r, v);
+    body(ch, v);
+  }
+}
+
+template <class C, class F>
+__device__ __forceinline__ void sweep(const C& c, F&& body) {
+  if (C::kAhead)
+    sweep_ahead(c.tm, c.nch(), body);
+  else
+    sweep_each(c.tm, c.nch(), body);
 }
 
 // Either row of a pair with its own width (key-row units, rows of two widths).
@@ -170,9 +194,11 @@ __device__ __forceinline__ constexpr uint32_t row_bytes_of(int dv) {
   return (uint32_t)dv * B / 8;
 }
 
-// Thread context of one item; FULL = compile-time 128 x 128 tile.
-template <bool FULL>
+// Thread context of one item; FULL = compile-time 128 x 128 tile; AHEAD: sweeps load the next
+// chunk while the current one is processed.
+template <bool FULL, bool AHEAD = true>
 struct Ctx {
+  static constexpr bool kAhead = AHEAD;
   int tid, warp, lane, dk_, dv_, nch_;
   bool act_;  // the lane's columns are < d_v
   uint32_t tm;
@@ -186,8 +212,8 @@ struct Ctx {
 
 // ---- pass A: exact codes into tensor memory, partial U and P ------------------------------
 // Head units of width B (16: fp16 head): rows in key order, row p at base + p * rb.
-template <int B, bool FULL>
-__device__ __forceinline__ void pass_a_head(const Ctx<FULL>& c, const uint8_t* blk) {
+template <int B, class C>
+__device__ __forceinline__ void pass_a_head(const C& c, const uint8_t* blk) {
   const int dv = c.dv();
   const uint32_t rb = row_bytes_of<B>(dv);
   const uint8_t* row0 = blk + (B == 16 ? 0u : 2u * (c.dk() + dv)) + (uint32_t)c.row0() * rb;
@@ -225,8 +251,8 @@ __device__ __forceinline__ void pass_a_head(const Ctx<FULL>& c, const uint8_t* b
 }
 
 // Key-row units: per-chunk width dispatch (rows are width-sorted), fp16 rows scaled by 1/c_j.
-template <bool FULL>
-__device__ __forceinline__ void pass_a_rows(const Ctx<FULL>& c, const uint8_t* blk, const float4& icv) {
+template <class C>
+__device__ __forceinline__ void pass_a_rows(const C& c, const uint8_t* blk, const float4& icv) {
   const float4* gkq = sp<float4>(S_GKQ) + c.row0() / 2;
   const uint4* rd4 = reinterpret_cast<const uint4*>(sp<uint32_t>(S_RD) + c.row0());
   float2 U[4], P[4];
@@ -286,8 +312,8 @@ __device__ __forceinline__ void pass_a_rows(const Ctx<FULL>& c, const uint8_t* b
 // it into their row factors.
 // KIND 0: quantized head (row maxima); 1: fp16 head (fp16 range check, no maxima); 2: key-row
 // units (row maxima; range check of the fp16 rows).
-template <int KIND, bool WS, bool TILDE, bool FULL>
-__device__ __forceinline__ void pass_b(const Ctx<FULL>& c, const float4& cv, const float4& bv,
+template <int KIND, bool WS, bool TILDE, class C>
+__device__ __forceinline__ void pass_b(const C& c, const float4& cv, const float4& bv,
                                        float* s_new) {
   const float2 cc[4] = {dup(cv.x), dup(cv.y), dup(cv.z), dup(cv.w)};
   const float2 bb[4] = {dup(bv.x), dup(bv.y), dup(bv.z), dup(bv.w)};
@@ -298,7 +324,7 @@ __device__ __forceinline__ void pass_b(const Ctx<FULL>& c, const float4& cv, con
   const uint4* rd4 = reinterpret_cast<const uint4*>(sp<uint32_t>(S_RD) + c.row0());
   const int dv = c.dv();
   bool of = false;
-  sweep(c.tm, c.nch(), [&](int ch, float2 (&v)[8]) {
+  sweep(c, [&](int ch, float2 (&v)[8]) {
     float rm[4];
 #pragma unroll
     for (int pr = 0; pr < 2; ++pr) {
@@ -354,8 +380,8 @@ __device__ __forceinline__ void pass_b(const Ctx<FULL>& c, const float4& cv, con
 // the tile row in the column passes; fp16 rows get r = w = 0. Returns the lane's r.
 // omega: this row's weight in the column passes, in (0, 1] (1 without an impact table): a row
 // weighted below 1 counts with w = fl(omega fl(1 / (r Q))), so it sets the column scales less.
-template <bool FULL>
-__device__ __forceinline__ float row_scales(const Ctx<FULL>& c, bool check, float omega) {
+template <class C>
+__device__ __forceinline__ float row_scales(const C& c, bool check, float omega) {
   const int p = c.row0() + c.lane;
   float r = 0.f, w = 0.f;
   if (p < c.dk()) {
@@ -367,7 +393,7 @@ __device__ __forceinline__ float row_scales(const Ctx<FULL>& c, bool check, floa
       const float rq = div_q(__fmul_rn(t, sp<float>(S_RT)[p]), Q, inv_q);  // exactly m / Q
       if (check && !(rq < 65520.f)) atomicOr(&c.flags[F_RANGE], 1);
       r = fminf(fmaxf(rq, kScaleFloor), 65504.f);
-      float wi = __frcp_rn(__fmul_rn(r, Q));
+      float wi = rcp_rn(__fmul_rn(r, Q));
       if (omega < 1.f) wi = __fmul_rn(omega, wi);
       w = __fmul_rn(t, wi);
     }
@@ -380,8 +406,8 @@ __device__ __forceinline__ float row_scales(const Ctx<FULL>& c, bool check, floa
 // After the last alternation of an impact-weighted fit, with S_RT holding the row maxima of
 // |S_ij| / c_j (row_pass with the final column scales): a row weighted below 1 widens its
 // scale to fit them, r = max(r, m / Q), so none of its codes leaves [-Q, Q]. Other rows keep r.
-template <bool FULL>
-__device__ __forceinline__ float row_refit(const Ctx<FULL>& c, float r, float omega) {
+template <class C>
+__device__ __forceinline__ float row_refit(const C& c, float r, float omega) {
   const int p = c.row0() + c.lane;
   if (p < c.dk() && omega < 1.f) {
     const int b = rd_width(sp<uint32_t>(S_RD)[p]);
@@ -397,11 +423,11 @@ __device__ __forceinline__ float row_refit(const Ctx<FULL>& c, float r, float om
 }
 
 // Column pass: max_i |S_ij| w_i over the warp's rows into red[warp].
-template <bool FULL>
-__device__ __forceinline__ void col_pass(const Ctx<FULL>& c, float* red) {
+template <class C>
+__device__ __forceinline__ void col_pass(const C& c, float* red) {
   const float2* w2 = reinterpret_cast<const float2*>(sp<float>(S_W) + c.row0());
   float m0[4] = {0.f, 0.f, 0.f, 0.f}, m1[4] = {0.f, 0.f, 0.f, 0.f};
-  sweep(c.tm, c.nch(), [&](int ch, float2 (&v)[8]) {
+  sweep(c, [&](int ch, float2 (&v)[8]) {
     const float2 wa = w2[2 * ch], wb = w2[2 * ch + 1];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
@@ -416,11 +442,11 @@ __device__ __forceinline__ void col_pass(const Ctx<FULL>& c, float* red) {
 }
 
 // Row pass of a later alternation: row maxima of |S_ij| v_j into S_RT.
-template <bool FULL>
-__device__ __forceinline__ void row_pass(const Ctx<FULL>& c, const float4& icv) {
+template <class C>
+__device__ __forceinline__ void row_pass(const C& c, const float4& icv) {
   const float2 ic[4] = {dup(icv.x), dup(icv.y), dup(icv.z), dup(icv.w)};
   float4* rt = reinterpret_cast<float4*>(sp<float>(S_RT) + c.row0());
-  sweep(c.tm, c.nch(), [&](int ch, float2 (&v)[8]) {
+  sweep(c, [&](int ch, float2 (&v)[8]) {
     float rm[4];
 #pragma unroll
     for (int pr = 0; pr < 2; ++pr) {
@@ -433,6 +459,51 @@ __device__ __forceinline__ void row_pass(const Ctx<FULL>& c, const float4& icv) 
     if (c.lane == 0) rt[ch] = make_float4(rm[0], rm[1], rm[2], rm[3]);
   });
   __syncwarp();
+}
+
+// ---- skipping the last column pass when it cannot change an fp16 column scale ----------------
+// The last column pass recomputes c'_j = max(max_i fl(|S_ij| w'_i), 2^-14) with the multipliers
+// w'_i of the last row pass, where the previous column pass used w_i. If every w'_i lies within a
+// factor (1 +- delta) of w_i, then c'_j lies within c_j (1 +- (delta + 2.1 u)), u = 2^-24 (each
+// product rounds once, and max and the floor are monotone). If that interval holds no fp16
+// rounding boundary, RN_fp16(c'_j) = RN_fp16(c_j), and the stored column scales (rounded once,
+// at the end) are exactly what the full pass would give. The row scales come from the last row
+// pass either way. So: warp 0 takes the slack of every column (its relative distance from c_j to
+// the nearest fp16 rounding boundary), every warp its largest relative change of w, and the pass
+// is skipped when the largest change stays below the smallest slack minus 2^-21 (> 2.1 u).
+
+// Relative distance from c (>= 2^-14, rounding to a normal fp16 value) to the nearest fp16
+// rounding boundary, rounded down; a value on a boundary gets 0.
+__device__ __forceinline__ float fp16_slack(float c) {
+  const __half h = __float2half_rn(c);
+  const unsigned short hb = __half_as_ushort(h);
+  const float hf = __half2float(h);
+  const float up = __half2float(__ushort_as_half((unsigned short)(hb + 1)));
+  const float dn = __half2float(__ushort_as_half((unsigned short)(hb - 1)));
+  const float mid_hi = 0.5f * (hf + up), mid_lo = 0.5f * (hf + dn);  // exact
+  const float dist = c <= kScaleFloor ? mid_hi - c : fminf(mid_hi - c, c - mid_lo);  // exact
+  return fmaxf(dist, 0.f) * rcp_approx(c) * (1.0f - 0x1p-20f);
+}
+
+// Warp 0: the smallest slack over the lane's four columns and the warp (all 128 columns), less
+// the margin, into S_FIT[4].
+__device__ __forceinline__ void column_slack(int warp, int lane, const float4& cm, bool act) {
+  if (warp != 0) return;
+  float t = act ? fminf(fminf(fp16_slack(cm.x), fp16_slack(cm.y)),
+                        fminf(fp16_slack(cm.z), fp16_slack(cm.w)))
+                : 1.f;
+  t = __uint_as_float(__reduce_min_sync(0xffffffffu, __float_as_uint(t)));  // t >= 0
+  if (lane == 0) sp<float>(S_FIT)[4] = t - 0x1p-21f;
+}
+
+// The lane's row: relative change of its column multiplier, rounded up (infinite when a zero
+// multiplier became nonzero); the warp's largest into S_FIT[warp].
+__device__ __forceinline__ void multiplier_change(int warp, int lane, float w_old, float w_new) {
+  float d = 0.f;
+  if (w_new != w_old) d = w_old > 0.f ? fabsf(w_new - w_old) * rcp_approx(w_old) * (1.0f + 0x1p-20f)
+                                      : __int_as_float(0x7f800000);
+  d = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(d)));  // d >= 0
+  if (lane == 0) sp<float>(S_FIT)[warp] = d;
 }
 
 // Max over the four warps' partial column maxima of the lane's columns, floored at 2^-14.
@@ -461,8 +532,8 @@ __device__ __forceinline__ float4 sum4(const float* red, int lane) {
 // Row scales: r16_i to the block (at the original row), t_i / r16_i into S_IR (t_i for fp16
 // rows); column scales: c16.
 // Returns the lane's correctly rounded 1/c16 of its four columns.
-template <bool FULL>
-__device__ __forceinline__ float4 store_scales(const Ctx<FULL>& c, uint8_t* dst, const float4& cm, float r) {
+template <class C>
+__device__ __forceinline__ float4 store_scales(const C& c, uint8_t* dst, const float4& cm, float r) {
   const int p = c.row0() + c.lane;
   if (p < c.dk()) {
     const uint32_t d = sp<uint32_t>(S_RD)[p];
@@ -520,8 +591,8 @@ __device__ __forceinline__ float magic_of() {
 }
 
 // Head units of width B.
-template <int B, bool FULL>
-__device__ __forceinline__ void requant_head(const Ctx<FULL>& c, uint8_t* dst, const float4& icv) {
+template <int B, class C>
+__device__ __forceinline__ void requant_head(const C& c, uint8_t* dst, const float4& icv) {
   const float2 ic[4] = {dup(icv.x), dup(icv.y), dup(icv.z), dup(icv.w)};
   const uint32_t rb = row_bytes_of<B>(c.dv());
   const float2* ir2 = reinterpret_cast<const float2*>(sp<float>(S_IR) + c.row0());
@@ -530,7 +601,7 @@ __device__ __forceinline__ void requant_head(const Ctx<FULL>& c, uint8_t* dst, c
   // the lane's bytes of the warp's first row (6-bit rows: the row start; store4<6> places them)
   uint8_t* base = dst + 2u * (c.dk() + c.dv()) + (uint32_t)c.row0() * rb +
                   (B == 6 ? 0u : (uint32_t)lane * (B / 2));
-  sweep(c.tm, c.nch(), [&](int ch, float2 (&v)[8]) {
+  sweep(c, [&](int ch, float2 (&v)[8]) {
     uint8_t* cb = base + (uint32_t)ch * 4u * rb;
 #pragma unroll
     for (int pr = 0; pr < 2; ++pr) {
@@ -587,8 +658,8 @@ __device__ __forceinline__ void requant_chunk_uniform(const float2 (&v)[8], cons
   }
 }
 
-template <bool FULL>
-__device__ __forceinline__ void requant_rows(const Ctx<FULL>& c, uint8_t* dst, const float4& icv) {
+template <class C>
+__device__ __forceinline__ void requant_rows(const C& c, uint8_t* dst, const float4& icv) {
   const float2 ic2[4] = {dup(icv.x), dup(icv.y), dup(icv.z), dup(icv.w)};
   const float ic[4] = {icv.x, icv.y, icv.z, icv.w};
   const float* irs = sp<float>(S_IR) + c.row0();
@@ -596,7 +667,7 @@ __device__ __forceinline__ void requant_rows(const Ctx<FULL>& c, uint8_t* dst, c
   const uint4* rd4 = reinterpret_cast<const uint4*>(sp<uint32_t>(S_RD) + c.row0());
   const bool act = c.act();
   const int lane = c.lane;
-  sweep(c.tm, c.nch(), [&](int ch, float2 (&v)[8]) {
+  sweep(c, [&](int ch, float2 (&v)[8]) {
     const uint4 d = rd4[ch];
     const uint32_t ds[4] = {d.x, d.y, d.z, d.w};
     const int b0 = rd_width(ds[0]);
@@ -619,13 +690,13 @@ __device__ __forceinline__ void requant_rows(const Ctx<FULL>& c, uint8_t* dst, c
 }
 
 // fp16 head: round and store the updated tile.
-template <bool FULL>
-__device__ __forceinline__ void store_pivot(const Ctx<FULL>& c, uint8_t* dst) {
+template <class C>
+__device__ __forceinline__ void store_pivot(const C& c, uint8_t* dst) {
   const uint32_t rb = 2u * c.dv();
   uint8_t* row0 = dst + (uint32_t)c.row0() * rb;
   const bool act = c.act();
   const int lane = c.lane;
-  sweep(c.tm, c.nch(), [&](int ch, float2 (&v)[8]) {
+  sweep(c, [&](int ch, float2 (&v)[8]) {
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
       const float2* g = v + 4 * (r >> 1);

@@ -79,7 +79,7 @@ __device__ __forceinline__ void fit_scales(const float (&S)[kRows][4], int fit_i
         if (Q > 0) {
           const float q = __fdiv_rn(tmp[lane], (float)Q);
           r = fmaxf(q, kScaleFloor);
-          w = __frcp_rn(__fmul_rn(r, (float)Q));
+          w = rcp_rn(__fmul_rn(r, (float)Q));
           if (omega && omega[i] < 1.f) w = __fmul_rn(omega[i], w);
         }
         rowR[i] = r;
@@ -110,7 +110,7 @@ __device__ __forceinline__ void fit_scales(const float (&S)[kRows][4], int fit_i
       for (int w = 0; w < kWarps; ++w) c = fmaxf(c, red[w * 2 * kMaxD + t]);
       c = fmaxf(c, kScaleFloor);
       col[COL_X * kMaxD + t] = c;
-      col[COL_INV * kMaxD + t] = __frcp_rn(c);
+      col[COL_INV * kMaxD + t] = rcp_rn(c);
     } else if (t < kMaxD) {  // columns past d_v: neutral values for the idle lanes
       col[COL_X * kMaxD + t] = kScaleFloor;
       col[COL_INV * kMaxD + t] = 1.f;

@@ -91,6 +91,7 @@ def lib() -> C.CDLL:
         "sq_debug_decode_step_fp32": [P, P, I32, P, P, P, P, P, P, P, P],
         "sq_allocate_bits": [I32, P, P, C.c_float, I32, P, P],
         "sq_debug_set_wait": [P, C.c_uint64, C.c_uint32],
+        "sq_debug_set_full_fit": [P, I32],
     }
     for name, args in sigs.items():
         fn = getattr(L, name)
@@ -204,6 +205,10 @@ def sq_debug_decode_step_fp32(pool: int, slot_idx: int, batch: int, q: int, k: i
 def sq_debug_set_wait(pool: int, wait_limit_ns: int, extra_expected_bytes: int) -> None:
     _chk(lib().sq_debug_set_wait(pool, int(wait_limit_ns), int(extra_expected_bytes)),
          "sq_debug_set_wait")
+
+
+def sq_debug_set_full_fit(pool: int, full_fit: int) -> None:
+    _chk(lib().sq_debug_set_full_fit(pool, int(full_fit)), "sq_debug_set_full_fit")
 
 
 def sq_window_flush(pool: int, slot_idx: int, n: int, stream: int) -> None:

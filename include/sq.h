@@ -287,6 +287,16 @@ SQ_API sq_status sq_debug_decode_step_fp32(sq_pool* pool, const int32_t* slot_id
 SQ_API sq_status sq_debug_set_wait(sq_pool* pool, uint64_t wait_limit_ns,
                                    uint32_t extra_expected_bytes);
 
+/*
+ * Test hook of the decode step's last column pass (the pages have no counterpart: it exists to
+ * check an exactness claim). The decode kernel skips the last column pass of the scale fit
+ * when a bound proves it cannot change any fp16 column scale (the multipliers of the last row
+ * pass moved less than every column scale's distance to an fp16 rounding boundary allows); the
+ * stored bytes are then exactly those of the full pass. full_fit = 1 makes every later decode
+ * step of this pool run the full pass, so a test can compare the two bit for bit; 0 restores
+ * the default. Host only. SQ_ERR_INVALID_ARG for a NULL pool or another value. */
+SQ_API sq_status sq_debug_set_full_fit(sq_pool* pool, int32_t full_fit);
+
 #ifdef __cplusplus
 }
 #endif

@@ -9,11 +9,17 @@
  *          1/x; y = fma(y0, fma(-x, y0, 1), y0). Checked against the correctly rounded
  *          reciprocal for every positive normal fp16 x, with y0 anywhere within 64 ulps of
  *          the true reciprocal (the hardware approximation is within one).
+ *  rcp32:  y = 1 / x for any single-precision x (24-bit significand) as y0 = an approximation
+ *          of 1/x, then two Newton steps in double precision, d = fma(d, fma(-x, d, 1), d)
+ *          from d = y0, and one rounding of d to single precision. Checked against the
+ *          correctly rounded reciprocal for every significand in [1, 2) at several exponents,
+ *          with y0 at 0, +-1, +-2 and +-64 ulps from the true reciprocal.
  *
  * The references round an exact double-precision quotient to single precision; that equals the
  * correctly rounded single-precision quotient because m / Q (Q odd) and 1 / x (x with an
  * 11-bit significand) never lie within 2^-36 (relative) of a single-precision rounding
- * midpoint, far more than double precision's 2^-53.
+ * midpoint, far more than double precision's 2^-53, and 1 / x for a 24-bit significand x never
+ * lies within 2^-49 of one (x times a 25-bit midpoint is never 1).
  *
  * Prints "div_mismatch=N rcp_mismatch=M cases=K". */
 #include <math.h>
@@ -58,6 +64,24 @@ int main(void) {
       if (bits_of(y) != bits_of(ref)) rcp_mis++;
     }
   }
-  printf("div_mismatch=%lld rcp_mismatch=%lld cases=%lld\n", div_mis, rcp_mis, cases);
+  long long rcp32_mis = 0;
+  const int rexps[5] = {-14, -3, 0, 6, 16};
+  const int offs[7] = {0, 1, -1, 2, -2, 64, -64};
+  for (int ei = 0; ei < 5; ++ei) {
+    for (uint32_t s = 0; s < (1u << 23); ++s) {
+      const float x = ldexpf(from_bits(0x3f800000u | s), rexps[ei]);
+      const float ref = (float)(1.0 / (double)x);
+      for (int k = 0; k < 7; ++k) {
+        const float y0 = from_bits(bits_of(ref) + (uint32_t)offs[k]);
+        double d = (double)y0;
+        d = fma(d, fma(-(double)x, d, 1.0), d);
+        d = fma(d, fma(-(double)x, d, 1.0), d);
+        cases++;
+        if (bits_of((float)d) != bits_of(ref)) rcp32_mis++;
+      }
+    }
+  }
+  printf("div_mismatch=%lld rcp_mismatch=%lld rcp32_mismatch=%lld cases=%lld\n", div_mis, rcp_mis,
+         rcp32_mis, cases);
   return 0;
 }

@@ -17,7 +17,7 @@ def lib():
 
 def test_exports_every_declared_symbol(lib):
     names = sq.exported_names()
-    assert len(names) == 17, names  # the calls include/sq.h declares
+    assert len(names) == 18, names  # the calls include/sq.h declares
     for n in names:
         assert hasattr(lib, n), n
 
@@ -93,3 +93,7 @@ def test_calls_on_null_pool_rejected(lib):
 
 def test_set_wait_rejects_a_null_pool(lib):
     assert lib.sq_debug_set_wait(None, 1000, 0) == sq.SQ_ERR_INVALID_ARG
+
+
+def test_set_full_fit_rejects_a_null_pool(lib):
+    assert lib.sq_debug_set_full_fit(None, 1) == sq.SQ_ERR_INVALID_ARG
