@@ -111,8 +111,12 @@ sq_status plan(const sq_layout* L, const uint8_t* bits, const uint8_t* pivot_mas
   P->max_head_bytes = maxb;
   if (L->unit == SQ_UNIT_KEY_ROW) {
     // Processing order of the decode kernel: each head's rows grouped by width (stable), so
-    // that row pairs and four-row chunks almost always share one width.
+    // that row pairs and four-row chunks almost always share one width; the four-row chunks of
+    // that sequence are then dealt to the warps in turn (warp w owns processing rows
+    // [32 w, 32 w + 32)), so every warp gets about the same mix of widths and none of them
+    // waits long for the others at the item's barriers.
     P->srows.assign((size_t)H * dk, 0);
+    const int n_ch = dk / 4, n_warps = (dk + 31) / 32;
     for (int h = 0; h < H; ++h) {
       std::vector<int> idx(dk);
       for (int i = 0; i < dk; ++i) idx[i] = i;
@@ -120,11 +124,25 @@ sq_status plan(const sq_layout* L, const uint8_t* bits, const uint8_t* pivot_mas
       std::stable_sort(idx.begin(), idx.end(), [&](int x, int y) {
         return sq::row_width(rt[x]) < sq::row_width(rt[y]);
       });
+      // chunk k of the sorted sequence goes to warp k % n_warps as its chunk k / n_warps; with
+      // d_k not a multiple of 32 the last warp owns fewer chunks, so the deal skips it once its
+      // chunks are full
+      std::vector<int> order;
+      order.reserve(dk);
+      std::vector<std::vector<int>> per_warp(n_warps);
+      int w = 0;
+      for (int k = 0; k < n_ch; ++k) {
+        for (int tries = 0; (int)per_warp[w].size() >= std::min(32, dk - 32 * w) && tries < n_warps; ++tries)
+          w = (w + 1) % n_warps;
+        for (int r = 0; r < 4; ++r) per_warp[w].push_back(idx[4 * k + r]);
+        w = (w + 1) % n_warps;
+      }
+      for (int ww = 0; ww < n_warps; ++ww) order.insert(order.end(), per_warp[ww].begin(), per_warp[ww].end());
       for (int p = 0; p < dk; ++p) {
-        const uint32_t d = rt[idx[p]];
+        const uint32_t d = rt[order[p]];
         if (sq::row_off(d) >= (1u << 16)) return SQ_ERR_INVALID_ARG;
         P->srows[(size_t)h * dk + p] =
-            (uint32_t)idx[p] << 24 | sq::row_off(d) << 8 | (uint32_t)sq::row_width(d);
+            (uint32_t)order[p] << 24 | sq::row_off(d) << 8 | (uint32_t)sq::row_width(d);
       }
     }
   }

@@ -303,13 +303,12 @@ __global__ void __launch_bounds__(kT, kMaxCtasPerSm) k_decode(const StepArgs a) 
     }
 
     // ---- refit: alternating row / column max-abs passes ----
-    // head units: every row factor A_i in [2^-60, 2^60] (key-row units keep the direct form,
-    // which makes their kernels smaller)
-    const bool tilde = !ROWS && !c.flags[F_BADA];
+    // the row-factored form when every row factor A_i is in [2^-60, 2^60], else the direct one
+    const bool tilde = !c.flags[F_BADA];
     if (tid < dk) sp<float>(S_TR)[tid] = tilde ? sp<float>(S_AK)[4 * (tid >> 1) + (tid & 1)] : 1.f;
     __syncwarp();
-    if (!ROWS && tilde)
-      pass_b<ROWS ? 2 : 0, WS, !ROWS>(c, cv, bv, s_new);
+    if (tilde)
+      pass_b<ROWS ? 2 : 0, WS, true>(c, cv, bv, s_new);
     else
       pass_b<ROWS ? 2 : 0, WS, false>(c, cv, bv, s_new);
     if (WS && a.update_only) {  // the refit and requantization run elsewhere
