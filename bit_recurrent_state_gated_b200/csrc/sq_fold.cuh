@@ -95,15 +95,21 @@ __device__ __forceinline__ void chunk_add(float2 (&v)[8], int r, int e, float ad
 // the chunk, the owner lane changes the element (x += add, or x = add), the warp stores it.
 // Returns the element's new value to the owner lane (0 elsewhere).
 template <class C>
-__device__ __forceinline__ float tile_patch(const C& c, int p, int j, float add, bool set) {
+__device__ __forceinline__ float tile_patch(const C& c, int p, int j, float add, bool set,
+                                            float* old = nullptr) {
   if (p / kRW != c.warp) return 0.f;  // warp-uniform
   const int ch = (p % kRW) / 4;
   uint32_t r[16];
   float2 v[8];
   tm_issue(c.tm + 16u * ch, r);
   tm_take(r, v);
-  float nv = 0.f;
+  float nv = 0.f, ov = 0.f;
   if (c.lane == j / 4) {
+#pragma unroll
+    for (int rr = 0; rr < 4; ++rr)
+#pragma unroll
+      for (int ee = 0; ee < 4; ++ee)
+        if (rr == p % 4 && ee == j % 4) ov = (rr & 1) ? v[4 * (rr >> 1) + ee].y : v[4 * (rr >> 1) + ee].x;
     chunk_add(v, p % 4, j % 4, add, set);
 #pragma unroll
     for (int rr = 0; rr < 4; ++rr)
@@ -113,6 +119,7 @@ __device__ __forceinline__ float tile_patch(const C& c, int p, int j, float add,
   }
   tmem_st16x2(c.tm + 16u * ch, v);
   tmem_wait_st();
+  if (old) *old = ov;
   return nv;
 }
 
@@ -185,12 +192,34 @@ __device__ __forceinline__ void window_fold(const Ctx<FULL>& c, const StepArgs& 
   __syncwarp();
   // ---- the frozen compensation entries: S_ij += g_i value (their code is 0) ----
   if (!pivot_head) {
+    bool lowered = false;  // a patch lowered the element that held the thread's maximum
     for (int o = 0; o < a.n_outliers; ++o) {
       const int idx = sp<int>(W_OE)[o];
       if (idx >= dk * dv) continue;
       const float pv = sp<float>(W_OE)[64 + o];
       const int i = idx / dv, j = idx % dv;
-      tmaxf = fmaxf(tmaxf, fabsf(tile_patch(c, sp<int>(W_INV)[i], j, sp<float>(W_GN)[i] * pv, false)));
+      float ov = 0.f;
+      const float nv = fabsf(tile_patch(c, sp<int>(W_INV)[i], j, sp<float>(W_GN)[i] * pv, false, &ov));
+      lowered |= nv < fabsf(ov) && fabsf(ov) >= tmaxf;
+      tmaxf = fmaxf(tmaxf, nv);
+    }
+    // then the recorded maximum may exceed every element of the thread: that warp rescans its
+    // tile, so that the thread maxima below are exact and the n-th largest of them bounds the
+    // n-th largest element from below
+    if (__any_sync(0xffffffffu, lowered)) {
+      tmaxf = 0.f;
+      sweep(c, [&](int ch, float2 (&v)[8]) {
+        if (ROWS) {
+          const uint4 d = rd4[ch];
+#pragma unroll
+          for (int r = 0; r < 4; ++r)
+            if (rd_width((&d.x)[r]) != 16)
+              tmaxf = fmaxf(tmaxf, (r & 1) ? rowmax_y(v + 4 * (r >> 1)) : rowmax_x(v + 4 * (r >> 1)));
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) tmaxf = max3abs(tmaxf, v[e].x, v[e].y);
+        }
+      });
     }
   }
   // ---- the n largest |S| of the quantized rows: fp16 compensation entries ----
@@ -256,10 +285,9 @@ __device__ __forceinline__ void window_fold(const Ctx<FULL>& c, const StepArgs& 
       }
     });
     __syncthreads();
-    // The thread maxima can exceed the tile's current values (an element changed by a frozen
-    // entry's patch after its maximum was taken), so the threshold may lie above the n-th
-    // largest element; then fewer than n candidates exist and the exact path below decides.
-    // With n or more candidates every element of the top n is among them.
+    // The thread maxima are exact (a warp whose patch lowered a thread's largest element
+    // rescanned above), so at least n elements reach the threshold and every element of the top
+    // n is among the candidates; the exact path below only serves more than kMaxCand ties.
     const int nc = misc[0];
     const bool ranked = nc >= n_out && nc <= kMaxCand;
     if (ranked) {
