@@ -316,10 +316,15 @@ __global__ void __launch_bounds__(kT, kMaxCtasPerSm) k_decode(const StepArgs a) 
       continue;
     }
     float r = row_scales(c, true, omega);
+    // the second (and last) alternation may be provably unable to change an fp16 scale (see
+    // row_scale_settled); not with row weights, whose closing refit needs the exact fp32 scales
+    const bool may_settle = a.fit_iters == 2 && !a.omega && !a.full_fit;
     col_pass(c, sp<float>(S_REDC));
-    __syncthreads();  // barrier 2
+    const bool unsettled_row = __syncthreads_or(may_settle && !row_scale_settled(r));  // barrier 2
     float4 cm = max4(sp<float>(S_REDC), c.lane);
-    for (int f = 1; f < a.fit_iters; ++f) {
+    const bool settled =  // the same in every warp: each holds every column scale
+        may_settle && !unsettled_row && __all_sync(0xffffffffu, !c.act() || column_scales_settled(cm));
+    for (int f = 1; f < a.fit_iters && !settled; ++f) {
       // the last column pass may be skipped (see column_slack); not with row weights, whose
       // closing refit needs the exact fp32 column scales
       const bool maybe_skip = f + 1 == a.fit_iters && !a.omega && !a.full_fit;

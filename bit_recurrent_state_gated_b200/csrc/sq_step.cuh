@@ -485,6 +485,31 @@ __device__ __forceinline__ float fp16_slack(float c) {
   return fmaxf(dist, 0.f) * rcp_approx(c) * (1.0f - 0x1p-20f);
 }
 
+// Distance of x's fp32 bit pattern from the nearest fp16 rounding boundary, in units of x's last
+// place: for x in the normal fp16 range the boundaries are exactly the fp32 values whose low 13
+// bits are 0x1000. Since x / ulp(x) < 2^24, a distance of d ulps is a relative distance above
+// d 2^-24.
+__device__ __forceinline__ int fp16_margin_ulps(float x) {
+  return abs((int)(__float_as_uint(x) & 0x1fffu) - 0x1000);
+}
+
+// Skipping the whole second alternation (fit_iters = 2) without looking at it. Following the
+// rounding chain of the rule (u = 2^-24; each operation rounds once; the row maxima m_i, the
+// column scales c_j <= (1 + u)^3 / (1 - u)^3, v_j = 1/c_j): the second row pass gives
+// m'_i in m_i [1 - 10 u, 1 + 8 u], hence r'_i in r_i [1 - 12 u, 1 + 10 u] for rows above the
+// 2^-14 floor (floored rows stay within [2^-14, 2^-14 (1 + 10 u)]), the multipliers
+// w'_i in w_i [1 - 16 u, 1 + 18 u], and the second column pass c'_j in c_j [1 - 18 u, 1 + 20 u].
+// So when every row scale lies more than 16 ulps and every column scale more than 24 ulps from
+// an fp16 rounding boundary (and no row scale is near the fp16 range's end), the second
+// alternation cannot change any fp16 scale: the stored bytes are those of the full fit.
+__device__ __forceinline__ bool row_scale_settled(float r) {
+  return r == 0.f || (r < 32768.f && fp16_margin_ulps(r) > 16);  // r == 0: an fp16 row
+}
+__device__ __forceinline__ bool column_scales_settled(const float4& cm) {
+  return fp16_margin_ulps(cm.x) > 24 && fp16_margin_ulps(cm.y) > 24 &&
+         fp16_margin_ulps(cm.z) > 24 && fp16_margin_ulps(cm.w) > 24;
+}
+
 // Warp 0: the smallest slack over the lane's four columns and the warp (all 128 columns), less
 // the margin, into S_FIT[4].
 __device__ __forceinline__ void column_slack(int warp, int lane, const float4& cm, bool act) {
