@@ -72,10 +72,11 @@ def algorithmic_bytes(wl: W.Workload, slot_bytes: int) -> dict:
     """Bytes one request-step must move (`total`): the packed state (codes, scales, fp16 units)
     read and written, q/k/v read, alpha/beta read, o written, the slot index read. Windowed
     layouts read the frozen block every token and write it once per window; the low-rank side
-    state they keep for the open window (the cumulative gate and one (k_hat, b) pair per token,
-    fp32) is this implementation's representation, not the method's bytes, so it is reported
-    apart as `side` and left out of `total`. A chunk of T tokens reads and writes the packed
-    state once: 1/T of it per request-step."""
+    state they keep for the open window (a header with the cumulative gate, one term per token:
+    the token's k in the I/O type and b / g in fp32 for the scalar gate; k / g and b in fp32 and
+    the per-row gates for the diagonal gate) is this implementation's representation, not the
+    method's bytes, so it is reported apart as `side` and left out of `total`. A chunk of T
+    tokens reads and writes the packed state once: 1/T of it per request-step."""
     esz = 2 if wl.io_dtype == W.IO_BF16 else 4
     H, dk, dv = wl.n_heads, wl.d_k, wl.d_v
     io = H * (2 * dk + dv) * esz + H * wl.alpha_width * 4 + H * 4 + H * dv * 4 + 4
@@ -86,11 +87,14 @@ def algorithmic_bytes(wl: W.Workload, slot_bytes: int) -> dict:
     else:
         Wn = wl.window
         state = slot_bytes + slot_bytes / Wn
-        term = 4 * (dk + dv)
-        # per head and window: token t reads t terms and (t > 0) the gate; tokens 0..W-2 write
-        # a term, the gate and the count
-        reads = sum(t * term + (4 * dk if t else 0) for t in range(Wn))
-        writes = (Wn - 1) * (term + 4 * dk + 4)
+        diag = wl.gate == W.GATE_DIAG
+        head = 16 + (4 * dk if diag else 0)  # header (count; scalar gate: g), diagonal: g [d_k]
+        kpart = 4 * dk if diag else (dk * esz + 15) // 16 * 16
+        term = kpart + 4 * dv
+        # per head and window: token t reads the header and t terms; tokens 0..W-2 write a
+        # term and the header (count and gate(s)); the last token folds and clears the count
+        reads = sum(head + t * term for t in range(Wn))
+        writes = (Wn - 1) * (dk * (4 if diag else esz) + 4 * dv + (4 + 4 * dk if diag else 8)) + 4
         side = H * (reads + writes) / Wn
     return {"state": state, "side": side, "io": io, "total": state + io}
 

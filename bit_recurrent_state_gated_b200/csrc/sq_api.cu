@@ -141,8 +141,13 @@ sq_status plan(const sq_layout* L, const uint8_t* bits, const uint8_t* pivot_mas
       for (int p = 0; p < dk; ++p) {
         const uint32_t d = rt[order[p]];
         if (sq::row_off(d) >= (1u << 16)) return SQ_ERR_INVALID_ARG;
-        P->srows[(size_t)h * dk + p] =
-            (uint32_t)order[p] << 24 | sq::row_off(d) << 8 | (uint32_t)sq::row_width(d);
+        const int p0 = p & ~3;  // the four-row chunk of processing row p
+        bool uniform = true;
+        for (int r = 1; r < 4; ++r)
+          uniform &= sq::row_width(rt[order[p0 + r]]) == sq::row_width(rt[order[p0]]);
+        P->srows[(size_t)h * dk + p] = (uint32_t)order[p] << 24 | sq::row_off(d) << 8 |
+                                       (uniform ? sq::kChunkUniform : 0u) |
+                                       (uint32_t)sq::row_width(d);
       }
     }
   }
@@ -154,9 +159,9 @@ sq_status plan(const sq_layout* L, const uint8_t* bits, const uint8_t* pivot_mas
   });
   if (L->window > 1) {
     if (L->window > 64) return SQ_ERR_INVALID_ARG;
-    // per (slot, head): token count (16-byte header), the cumulative gate g (d_k fp32) and
-    // `window` low-rank terms (k_hat [d_k], b [d_v] fp32)
-    P->side_head_bytes = 16 + 4u * (size_t)dk + (size_t)L->window * 4u * (size_t)(dk + dv);
+    // per (slot, head): header, cumulative gate(s) and `window` low-rank terms (sq::SideFmt)
+    const sq::SideFmt f(dk, dv, L->gate, L->io_dtype);
+    P->side_head_bytes = f.head + (size_t)L->window * f.stride;
     P->side_head_bytes = (P->side_head_bytes + 15) / 16 * 16;
     P->side_slot_bytes = (size_t)H * P->side_head_bytes;
     P->side_slot_bytes = (P->side_slot_bytes + 255) / 256 * 256;
@@ -451,7 +456,7 @@ sq_status sq_window_flush(sq_pool* pool, const int32_t* slot_idx, int32_t n, voi
   if (!slot_idx || !aligned(slot_idx, 4)) return SQ_ERR_INVALID_ARG;
   const sq::StepArgs a = step_args(pool, slot_idx, n, nullptr, nullptr, nullptr, nullptr,
                                    nullptr, nullptr, nullptr);
-  return cuda_status(sq::launch_window_flush(a, pool->num_sms, static_cast<cudaStream_t>(stream)));
+  return cuda_status(sq::launch_window_flush(a, pool->L.gate, pool->L.io_dtype, static_cast<cudaStream_t>(stream)));
 }
 
 sq_status sq_pool_set_row_impact(sq_pool* pool, const float* impact) {

@@ -432,15 +432,15 @@ __global__ void __launch_bounds__(kT, ROWS ? 4 : 3) k_chunk(const StepArgs a) {
       fetch_meta(next_meta);
     }
     if (skip) {
-      if (tid == 0)
-        if (tid == 0) atomicOr(a.flag, hdr.valid ? SQ_FLAG_NONFINITE_BIT : SQ_FLAG_BAD_SLOT_BIT);
+      if (tid == 0) atomicOr(a.flag, hdr.valid ? SQ_FLAG_NONFINITE_BIT : SQ_FLAG_BAD_SLOT_BIT);
       for (int x = tid; x < T * dv; x += kT) a.out[(size_t)io * T * dv + x] = __int_as_float(0x7fc00000);
     } else {  // fold the chunk into the block
       float4 bv = make_float4(0.f, 0.f, 0.f, 0.f);
       if (c.act()) bv = *reinterpret_cast<const float4*>(sp<float>(W_OU) + 4 * c.lane);
       uint8_t* dst = a.pool + (size_t)hdr.slot * a.slot_bytes + hdr.off;
-      window_fold<GATE, FULL, ROWS>(c, a, blk, terms, T - 1 - t0, mode, cv, bv, dst, omega,
-                                    &dummy_count);
+      window_fold<GATE, FULL, ROWS, false>(c, a, blk, reinterpret_cast<const uint8_t*>(terms),
+                                           4u * (uint32_t)(dk + dv), 4u * (uint32_t)dk,
+                                           T - 1 - t0, mode, cv, bv, dst, omega, &dummy_count);
     }
     __syncthreads();
   }

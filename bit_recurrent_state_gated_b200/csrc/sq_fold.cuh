@@ -22,10 +22,11 @@ namespace {
 // token), takes the n largest |S| of the quantized rows as fp16 compensation entries, and runs
 // the per-step kernel's fit and requantize passes on the rest.
 //
-// Side block of one (slot, head): int32 count | pad to 16 B | g [d_k] fp32 |
-// (W - 1) x (k_hat [d_k] fp32, b [d_v] fp32). Two stages hold the next items' q, k, v
-// (alpha, row table), side header + g and frozen block; the low-rank terms, whose count is known
-// only once the header has landed, follow into their own buffer while pass A runs.
+// Side block of one (slot, head): see SideFmt (sq_internal.h); for the scalar gate a term holds
+// the token's k in the I/O type and b_s / g_s, whose product is k_hat_s b_s^T. Two stages hold
+// the next items' q, k, v (alpha, row table), side header (+ g) and frozen block; the low-rank
+// terms, whose count is known only once the header has landed, follow into their own buffer
+// while pass A runs.
 // =============================================================================================
 constexpr int kMaxWin = 64;
 constexpr int kMaxCand = 256;  // candidate entries for the compensation choice
@@ -62,8 +63,10 @@ enum { F_UNDER = 2 };
 // low-rank term buffer and the head table.
 struct WDPlan {
   uint32_t esz, k_off, q_off, v_off, al_off, rt_off, sh_off, blk_off, stage, terms, tab, total;
+  SideFmt side;
   __host__ __device__ WDPlan(int dk, int dv, int io, int gate, int per_row, uint32_t stage_bytes,
-                             int n_heads, int window) {
+                             int n_heads, int window)
+      : side(dk, dv, gate, io) {
     esz = io == 1 ? 2u : 4u;
     k_off = (uint32_t)sizeof(StageHdr);
     q_off = k_off + dk * esz;
@@ -71,13 +74,28 @@ struct WDPlan {
     al_off = v_off + dv * esz;
     rt_off = al_off + (gate == 1 ? 4u * dk : 0u);
     sh_off = rt_off + (per_row ? 4u * dk : 0u);
-    blk_off = sh_off + 16u + 4u * dk;
+    blk_off = sh_off + side.head;
     stage = blk_off + round16(stage_bytes + kSlack);
     terms = W_STAGE + 2u * stage;
-    tab = terms + (uint32_t)(window - 1) * 4u * (dk + dv);
+    tab = terms + (uint32_t)(window - 1) * side.stride;
     total = tab + round16(20u * (uint32_t)n_heads);
   }
 };
+
+// The k part of four rows of a term: fp32, or bf16 (K16); head units' four rows are consecutive
+// (one load), key-row units' are gathered by original row.
+template <bool K16, bool ROWS>
+__device__ __forceinline__ float4 term_k4(const uint8_t* t, const int (&orow)[4]) {
+  if (K16) {
+    if (ROWS) return make_float4(ld_io(t, 1, orow[0]), ld_io(t, 1, orow[1]), ld_io(t, 1, orow[2]), ld_io(t, 1, orow[3]));
+    const uint2 w = *reinterpret_cast<const uint2*>(reinterpret_cast<const uint16_t*>(t) + orow[0]);
+    return make_float4(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xffff0000u),
+                       __uint_as_float(w.y << 16), __uint_as_float(w.y & 0xffff0000u));
+  }
+  const float* k = reinterpret_cast<const float*>(t);
+  if (ROWS) return make_float4(k[orow[0]], k[orow[1]], k[orow[2]], k[orow[3]]);
+  return *reinterpret_cast<const float4*>(k + orow[0]);
+}
 
 // Add `add` to element (row r of the chunk, column e) of the pairs v (r, e uniform or not).
 __device__ __forceinline__ void chunk_add(float2 (&v)[8], int r, int e, float add, bool set) {
@@ -127,15 +145,16 @@ __device__ __forceinline__ float tile_patch(const C& c, int p, int j, float add,
 __device__ __forceinline__ uint32_t wkey(float v) { return (__float_as_uint(v) & 0x7fffffffu) + 1u; }
 
 // The fold at the window's end (all threads). v of the lane's columns: cv (old c16), bv (b).
-template <int GATE, bool FULL, bool ROWS>
+// terms: cnt terms of `tstride` bytes, the k part (bf16 if K16, else fp32) then at `boff` the b
+// part, fp32; each contributes the rank-one product of its parts.
+template <int GATE, bool FULL, bool ROWS, bool K16>
 __device__ __forceinline__ void window_fold(const Ctx<FULL>& c, const StepArgs& a, const uint8_t* blk,
-                                            const float* terms, int cnt, int mode,
-                                            const float4& cv, const float4& bv, uint8_t* dst,
-                                            float omega, int32_t* count) {
+                                            const uint8_t* terms, uint32_t tstride, uint32_t boff,
+                                            int cnt, int mode, const float4& cv, const float4& bv,
+                                            uint8_t* dst, float omega, int32_t* count) {
   const int dk = c.dk(), dv = c.dv(), tid = c.tid, lane = c.lane;
   const bool pivot_head = !ROWS && mode == MODE_PIVOT;
   const int n_out = pivot_head ? 0 : a.n_outliers;
-  const uint32_t ts = (uint32_t)(dk + dv);
   const float2 cc[4] = {dup(cv.x), dup(cv.y), dup(cv.z), dup(cv.w)};
   const float2 bb[4] = {dup(bv.x), dup(bv.y), dup(bv.z), dup(bv.w)};
   const float4* ak = sp<float4>(S_AK) + c.row0() / 2;
@@ -156,15 +175,11 @@ __device__ __forceinline__ void window_fold(const Ctx<FULL>& c, const StepArgs& 
     }
 #pragma unroll 1
     for (int s = 0; s < cnt; ++s) {
-      const float* t = terms + (size_t)s * ts;
-      const float4 b4 = c.act() ? *reinterpret_cast<const float4*>(t + dk + 4 * lane)
+      const uint8_t* t = terms + (size_t)s * tstride;
+      const float4 b4 = c.act() ? reinterpret_cast<const float4*>(t + boff)[lane]
                                 : make_float4(0.f, 0.f, 0.f, 0.f);
       const float2 bs[4] = {dup(b4.x), dup(b4.y), dup(b4.z), dup(b4.w)};
-      float4 k4;  // k_hat of the chunk's four rows (head units: rows 4ch..4ch+3, one load)
-      if (ROWS)
-        k4 = make_float4(t[orow[0]], t[orow[1]], t[orow[2]], t[orow[3]]);
-      else
-        k4 = *reinterpret_cast<const float4*>(t + orow[0]);
+      const float4 k4 = term_k4<K16, ROWS>(t, orow);  // the chunk's four rows
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         acc[e] = __ffma2_rn(lo(k4), bs[e], acc[e]);
@@ -417,9 +432,8 @@ __device__ __forceinline__ void window_fold(const Ctx<FULL>& c, const StepArgs& 
     if (tid == 0) *count = 0;
     return;
   }
-  {  // row maxima (fp16 rows: range check)
+  {  // row maxima (row_scales checks the fp16 rows' range on them)
     float4* rtab = reinterpret_cast<float4*>(sp<float>(S_RT) + c.row0());
-    bool of = false;
     sweep(c, [&](int ch, float2 (&v)[8]) {
       float rm[4];
 #pragma unroll
@@ -428,15 +442,7 @@ __device__ __forceinline__ void window_fold(const Ctx<FULL>& c, const StepArgs& 
         rm[2 * pr + 1] = warp_max_nonneg(rowmax_y(v + 4 * pr));
       }
       if (lane == 0) rtab[ch] = make_float4(rm[0], rm[1], rm[2], rm[3]);
-      if (ROWS) {
-        const uint4 d = rd4[ch];
-        const uint32_t ds[4] = {d.x, d.y, d.z, d.w};
-#pragma unroll
-        for (int r = 0; r < 4; ++r)
-          if (rd_width(ds[r]) == 16 && !(rm[r] < 65520.f)) of = true;
-      }
     });
-    if (of) atomicOr(&c.flags[F_RANGE], 1);
     __syncwarp();
   }
   float r = row_scales(c, true, omega);

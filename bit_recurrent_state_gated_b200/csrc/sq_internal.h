@@ -27,6 +27,27 @@ struct HeadDesc {
 // width 16 for an fp16 pivot row.
 __host__ __device__ inline uint32_t row_off(uint32_t d) { return d >> 8; }
 __host__ __device__ inline int row_width(uint32_t d) { return (int)(d & 0xff); }
+// Key-row units' processing-order descriptors carry this bit when their four-row chunk has one
+// width.
+constexpr uint32_t kChunkUniform = 0x80u;
+
+// Windowed variant: the side block of one (slot, head) holds a 16-byte header (int32 token
+// count; for the scalar gate the cumulative gate g, fp32, at byte 4), for the diagonal gate the
+// cumulative gates g [d_k] fp32, then up to `window` low-rank terms. A term is a k part, then a
+// b part [d_v] fp32. Scalar gate: the token's own k in the I/O type and b / g_s, since
+// b (k_hat . y) = (b / g_s)(k . y) with k_hat = k / g_s; diagonal gate: k_hat in fp32 and b.
+struct SideFmt {
+  uint32_t head;    // bytes before the first term
+  uint32_t kbytes;  // k part of a term, a multiple of 16
+  uint32_t stride;  // bytes of a term
+  bool k16;         // k part in bf16
+  __host__ __device__ SideFmt(int dk, int dv, int gate, int io) {
+    k16 = gate == 0 && io == 1;
+    head = gate == 1 ? 16u + 4u * (uint32_t)dk : 16u;
+    kbytes = gate == 1 ? 4u * (uint32_t)dk : ((uint32_t)dk * (io == 1 ? 2u : 4u) + 15u) / 16u * 16u;
+    stride = kbytes + 4u * (uint32_t)dv;
+  }
+};
 
 struct StepArgs {
   uint8_t* pool;
@@ -91,7 +112,7 @@ cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t st);
 cudaError_t launch_dequantize(const QuantArgs& a, cudaStream_t st);
 cudaError_t launch_window_step(const StepArgs& a, int gate, int io, int num_sms,
                                cudaStream_t st);
-cudaError_t launch_window_flush(const StepArgs& a, int num_sms, cudaStream_t st);
+cudaError_t launch_window_flush(const StepArgs& a, int gate, int io, cudaStream_t st);
 cudaError_t launch_chunk(const StepArgs& a, int gate, int io, int num_sms, cudaStream_t st);
 // Heads and tile shape of a pool (for entry points outside the pool's own file).
 void pool_dims(const sq_pool* p, int* n_heads, int* d_k, int* d_v);

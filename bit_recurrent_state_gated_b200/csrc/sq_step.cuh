@@ -67,10 +67,13 @@ constexpr uint32_t S_FIT = S_TR + 512;        // [4] per-warp change of the colu
 constexpr uint32_t S_STAGE = S_FIT + 32;      // staging buffer, then the head table
 static_assert(S_STAGE % 16 == 0 && S_GKQ % 16 == 0 && S_REDU % 16 == 0, "16-byte aligned");
 
-// Row descriptor, processing order: original row << 24 | byte offset in the block << 8 | width.
+// Row descriptor, processing order: original row << 24 | byte offset in the block << 8 |
+// uniform << 7 | width, where the uniform bit marks every row of a key-row unit's four-row chunk
+// whose rows share one width (set when the pool is made).
 __device__ __forceinline__ int rd_row(uint32_t d) { return (int)(d >> 24); }
 __device__ __forceinline__ uint32_t rd_off(uint32_t d) { return (d >> 8) & 0xffffu; }
-__device__ __forceinline__ int rd_width(uint32_t d) { return (int)(d & 0xffu); }
+__device__ __forceinline__ int rd_width(uint32_t d) { return (int)(d & 0x1fu); }
+__device__ __forceinline__ bool rd_uniform(uint32_t d) { return (d & 0x80u) != 0u; }
 
 // Stage: header, k, q, v, (alpha), (row table), head block.
 struct DPlan {
@@ -250,7 +253,37 @@ __device__ __forceinline__ void pass_a_head(const C& c, const uint8_t* blk) {
       make_float4(P[0].x + P[0].y, P[1].x + P[1].y, P[2].x + P[2].y, P[3].x + P[3].y);
 }
 
-// Key-row units: per-chunk width dispatch (rows are width-sorted), fp16 rows scaled by 1/c_j.
+// Key-row units: one width dispatch per chunk whose four rows share a width (the uniform bit),
+// per row pair otherwise; fp16 rows are scaled by 1/c_j.
+__device__ __forceinline__ void unpack_pair_rt(uint32_t da, uint32_t db, const uint8_t* blk,
+                                               int lane, const float (&ic)[4], float2 (&x)[4]) {
+  const int wa = rd_width(da), wb = rd_width(db);
+  const uint8_t* ra = blk + rd_off(da);
+  const uint8_t* rbp = blk + rd_off(db);
+  if (wa == wb) {
+    switch (wa) {
+      case 2: unpack_pair<2>(ra, rbp, lane, x); break;
+      case 4: unpack_pair<4>(ra, rbp, lane, x); break;
+      case 6: unpack_pair<6>(ra, rbp, lane, x); break;
+      case 8: unpack_pair<8>(ra, rbp, lane, x); break;
+      default: unpack_pair<16>(ra, rbp, lane, x); break;
+    }
+  } else {
+    unpack_mixed(wa, ra, wb, rbp, lane, x);
+  }
+  if (wa == 16 || wb == 16) {  // fp16 rows hold values: x = value / c_j
+#pragma unroll
+    for (int e = 0; e < 4; ++e) x[e] = f2(wa == 16 ? x[e].x * ic[e] : x[e].x, wb == 16 ? x[e].y * ic[e] : x[e].y);
+  }
+}
+
+template <int B>
+__device__ __forceinline__ void unpack_chunk(const uint4& d, const uint8_t* blk, int lane,
+                                             float2 (&x0)[4], float2 (&x1)[4]) {
+  unpack_pair<B>(blk + rd_off(d.x), blk + rd_off(d.y), lane, x0);
+  unpack_pair<B>(blk + rd_off(d.z), blk + rd_off(d.w), lane, x1);
+}
+
 template <class C>
 __device__ __forceinline__ void pass_a_rows(const C& c, const uint8_t* blk, const float4& icv) {
   const float4* gkq = sp<float4>(S_GKQ) + c.row0() / 2;
@@ -262,40 +295,39 @@ __device__ __forceinline__ void pass_a_rows(const C& c, const uint8_t* blk, cons
 #pragma unroll 1
   for (int ch = 0; ch < c.nch(); ++ch) {
     const uint4 d = rd4[ch];
-    const uint32_t ds[4] = {d.x, d.y, d.z, d.w};
+    float2 x0[4], x1[4];
+    if (!c.act()) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) x0[e] = x1[e] = f2(0.f, 0.f);
+    } else if (rd_uniform(d.x)) {
+      switch (rd_width(d.x)) {
+        case 2: unpack_chunk<2>(d, blk, c.lane, x0, x1); break;
+        case 4: unpack_chunk<4>(d, blk, c.lane, x0, x1); break;
+        case 6: unpack_chunk<6>(d, blk, c.lane, x0, x1); break;
+        case 8: unpack_chunk<8>(d, blk, c.lane, x0, x1); break;
+        default:  // fp16 rows hold values: x = value / c_j
+          unpack_chunk<16>(d, blk, c.lane, x0, x1);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            x0[e] = __fmul2_rn(x0[e], dup(ic[e]));
+            x1[e] = __fmul2_rn(x1[e], dup(ic[e]));
+          }
+          break;
+      }
+    } else {
+      unpack_pair_rt(d.x, d.y, blk, c.lane, ic, x0);
+      unpack_pair_rt(d.z, d.w, blk, c.lane, ic, x1);
+    }
+    const float4 g0 = gkq[2 * ch], g1 = gkq[2 * ch + 1];
     float2 v[8];
 #pragma unroll
-    for (int pr = 0; pr < 2; ++pr) {
-      const uint32_t da = ds[2 * pr], db = ds[2 * pr + 1];
-      const int wa = rd_width(da), wb = rd_width(db);
-      const uint8_t* ra = blk + rd_off(da);
-      const uint8_t* rbp = blk + rd_off(db);
-      float2 x[4];
-      if (!c.act()) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) x[e] = f2(0.f, 0.f);
-      } else if (wa == wb) {
-        switch (wa) {
-          case 2: unpack_pair<2>(ra, rbp, c.lane, x); break;
-          case 4: unpack_pair<4>(ra, rbp, c.lane, x); break;
-          case 6: unpack_pair<6>(ra, rbp, c.lane, x); break;
-          case 8: unpack_pair<8>(ra, rbp, c.lane, x); break;
-          default: unpack_pair<16>(ra, rbp, c.lane, x); break;
-        }
-      } else {
-        unpack_mixed(wa, ra, wb, rbp, c.lane, x);
-      }
-      if (wa == 16 || wb == 16) {  // fp16 rows hold values: x = value / c_j
-#pragma unroll
-        for (int e = 0; e < 4; ++e) x[e] = f2(wa == 16 ? x[e].x * ic[e] : x[e].x, wb == 16 ? x[e].y * ic[e] : x[e].y);
-      }
-      const float4 g = gkq[2 * ch + pr];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        U[e] = __ffma2_rn(x[e], lo(g), U[e]);
-        P[e] = __ffma2_rn(x[e], hi(g), P[e]);
-        v[4 * pr + e] = x[e];
-      }
+    for (int e = 0; e < 4; ++e) {
+      U[e] = __ffma2_rn(x0[e], lo(g0), U[e]);
+      P[e] = __ffma2_rn(x0[e], hi(g0), P[e]);
+      U[e] = __ffma2_rn(x1[e], lo(g1), U[e]);
+      P[e] = __ffma2_rn(x1[e], hi(g1), P[e]);
+      v[e] = x0[e];
+      v[4 + e] = x1[e];
     }
     tmem_st16x2(c.tm + 16u * ch, v);
   }
@@ -311,7 +343,7 @@ __device__ __forceinline__ void pass_a_rows(const C& c, const uint8_t* blk, cons
 // row factor t_i (A_i or 1) by which a tile row is the state; the fit and the requantization take
 // it into their row factors.
 // KIND 0: quantized head (row maxima); 1: fp16 head (fp16 range check, no maxima); 2: key-row
-// units (row maxima; range check of the fp16 rows).
+// units (row maxima; row_scales checks the fp16 rows' range on them).
 template <int KIND, bool WS, bool TILDE, class C>
 __device__ __forceinline__ void pass_b(const C& c, const float4& cv, const float4& bv,
                                        float* s_new) {
@@ -350,7 +382,7 @@ __device__ __forceinline__ void pass_b(const C& c, const float4& cv, const float
       of |= !(m < 65520.f);
     }
     if (KIND != 1 && c.lane == 0) rt[ch] = make_float4(rm[0], rm[1], rm[2], rm[3]);
-    if (KIND == 2 || WS) {
+    if (WS) {
       const uint4 d = rd4[ch];
       const uint32_t ds[4] = {d.x, d.y, d.z, d.w};
       const float4 t4 = tr4[ch];
@@ -361,9 +393,7 @@ __device__ __forceinline__ void pass_b(const C& c, const float4& cv, const float
         const float t = KIND == 1 ? 1.f : ts[r];
         const float4 row = (r & 1) ? make_float4(g[0].y, g[1].y, g[2].y, g[3].y)
                                    : make_float4(g[0].x, g[1].x, g[2].x, g[3].x);
-        if (KIND == 2 && rd_width(ds[r]) == 16 && c.act())  // |t x| < 65520
-          of |= !(t * fmaxf(max3abs(row.x, row.y, row.z), fabsf(row.w)) < 65520.f);
-        if (WS && c.act())
+        if (c.act())
           *reinterpret_cast<float4*>(s_new + (size_t)rd_row(ds[r]) * dv + 4 * c.lane) =
               make_float4(t * row.x, t * row.y, t * row.z, t * row.w);
       }
@@ -377,7 +407,8 @@ __device__ __forceinline__ void pass_b(const C& c, const float4& cv, const float
 
 // Row scales from the row maxima in S_RT, one row per lane: m = t max |tile row|,
 // r = max(m / Q, 2^-14) (at most the largest fp16), w = 1 / (r Q); S_W gets t w, the factor of
-// the tile row in the column passes; fp16 rows get r = w = 0. Returns the lane's r.
+// the tile row in the column passes; fp16 rows get r = w = 0, and with `check` their values
+// must round to finite fp16 (m < 65520). Returns the lane's r.
 // omega: this row's weight in the column passes, in (0, 1] (1 without an impact table): a row
 // weighted below 1 counts with w = fl(omega fl(1 / (r Q))), so it sets the column scales less.
 template <class C>
@@ -396,6 +427,8 @@ __device__ __forceinline__ float row_scales(const C& c, bool check, float omega)
       float wi = rcp_rn(__fmul_rn(r, Q));
       if (omega < 1.f) wi = __fmul_rn(omega, wi);
       w = __fmul_rn(t, wi);
+    } else if (check && !(__fmul_rn(sp<float>(S_TR)[p], sp<float>(S_RT)[p]) < 65520.f)) {
+      atomicOr(&c.flags[F_RANGE], 1);
     }
   }
   sp<float>(S_W)[p] = w;
@@ -696,7 +729,7 @@ __device__ __forceinline__ void requant_rows(const C& c, uint8_t* dst, const flo
     const uint4 d = rd4[ch];
     const uint32_t ds[4] = {d.x, d.y, d.z, d.w};
     const int b0 = rd_width(ds[0]);
-    const bool uni = b0 == rd_width(ds[1]) && b0 == rd_width(ds[2]) && b0 == rd_width(ds[3]);
+    const bool uni = rd_uniform(ds[0]);
     if (uni && b0 == 2) {
       requant_chunk_uniform<2>(v, ds, dst, ir2, ch, ic2, lane, act);
     } else if (uni && b0 == 4) {

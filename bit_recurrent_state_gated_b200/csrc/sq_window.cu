@@ -14,8 +14,8 @@
 // token the state is materialized, the compensation entries are chosen, and it is refit and
 // requantized (sq_tile.cuh), as in the per-step path.
 //
-// Side block of one (slot, head): int32 count | pad to 16 B | g [d_k] fp32 |
-// W x (k_hat [d_k] fp32, b [d_v] fp32).
+// Side block of one (slot, head): see SideFmt (sq_internal.h). For the scalar gate a term holds
+// the token's k and b / g_s, whose product is the same rank-one term k_hat_s b_s^T.
 #include "sq_pair.cuh"
 #include "sq_tile.cuh"
 
@@ -99,7 +99,7 @@ __device__ __forceinline__ void flush_tile(const StepArgs& a, TileSmem& ts, cons
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, dk = a.dk, dv = a.dv;
   float S[kRows][4];
   frozen_tile<true>(S, blk, hd, rows, a.n_outliers, warp, lane, dk, dv);
-  const int tstride = dk + dv;
+  const int tstride = dk + dv;  // terms: k part [d_k], b part [d_v], fp32
   if (4 * lane < dv) {
     for (int t = 0; t < nterms; ++t) {
       const float* kh = terms + (size_t)t * tstride;
@@ -137,7 +137,7 @@ __device__ __forceinline__ void flush_tile(const StepArgs& a, TileSmem& ts, cons
 }
 
 // Fold each listed slot's open window into its block now (no-op at count 0).
-__global__ void __launch_bounds__(kThreads) k_window_flush(const StepArgs a) {
+__global__ void __launch_bounds__(kThreads) k_window_flush(const StepArgs a, int gate, int io) {
   extern __shared__ __align__(16) uint8_t dyn[];
   __shared__ WSmem sm;
   const int tid = threadIdx.x, dk = a.dk, dv = a.dv, H = a.H, W = a.window;
@@ -157,8 +157,20 @@ __global__ void __launch_bounds__(kThreads) k_window_flush(const StepArgs a) {
   uint8_t* blk = dyn;
   float* terms = reinterpret_cast<float*>(dyn + round16(a.stage_bytes + kSlack));
   copy16(blk, dst, hd.bytes, a.flag);
-  copy16(terms, side + 16 + 4 * dk, (uint32_t)cnt * (dk + dv) * 4, a.flag);
-  copy16(sm.g, side + 16, dk * 4, a.flag);
+  const SideFmt f(dk, dv, gate, io);
+  if (gate == 1) {  // the terms as stored: k_hat and b, fp32
+    copy16(terms, side + f.head, (uint32_t)cnt * f.stride, a.flag);
+    copy16(sm.g, side + 16, dk * 4, a.flag);
+  } else {  // the token's k (I/O type) and b / g_s, to fp32 terms; one gate for every row
+    for (int x = tid; x < cnt * (dk + dv); x += kThreads) {
+      const int t = x / (dk + dv), e = x % (dk + dv);
+      const uint8_t* tp = side + f.head + (size_t)t * f.stride;
+      terms[x] = e >= dk ? reinterpret_cast<const float*>(tp + f.kbytes)[e - dk]
+                         : f.k16 ? __uint_as_float((uint32_t)reinterpret_cast<const uint16_t*>(tp)[e] << 16)
+                                 : reinterpret_cast<const float*>(tp)[e];
+    }
+    for (int i = tid; i < dk; i += kThreads) sm.g[i] = reinterpret_cast<const float*>(side)[1];
+  }
   __syncthreads();
   flush_tile(a, sm.t, blk, terms, cnt, sm.g, false, nullptr, nullptr, dst, hd, rows,
              a.omega ? a.omega + (size_t)h * dk : nullptr, count);
@@ -167,14 +179,14 @@ __global__ void __launch_bounds__(kThreads) k_window_flush(const StepArgs a) {
 
 }  // namespace
 
-cudaError_t launch_window_flush(const StepArgs& a, int, cudaStream_t st) {
+cudaError_t launch_window_flush(const StepArgs& a, int gate, int io, cudaStream_t st) {
   if (a.window > kMaxWindow) return cudaErrorInvalidValue;
   const int items = a.batch * a.H;
   if (items < 1) return cudaSuccess;
   const uint32_t dyn = round16(a.stage_bytes + kSlack) + (uint32_t)a.window * (a.dk + a.dv) * 4;
   cudaError_t e = cudaFuncSetAttribute(k_window_flush, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
   if (e != cudaSuccess) return e;
-  k_window_flush<<<items, kThreads, dyn, st>>>(a);
+  k_window_flush<<<items, kThreads, dyn, st>>>(a, gate, io);
   return cudaGetLastError();
 }
 

@@ -24,8 +24,8 @@ __global__ void __launch_bounds__(kT, 3) k_window(const StepArgs a) {
   const int H = a.H, B = a.batch, dk = c.dk(), dv = c.dv(), tid = c.tid, W = a.window;
   const int n_items = B * H;
   const int stride = gridDim.x;
-  const uint32_t tbytes = 4u * (uint32_t)(dk + dv);
-  float* terms = reinterpret_cast<float*>(smem + P.terms);
+  const uint32_t tbytes = P.side.stride, kbytes = P.side.kbytes;
+  uint8_t* terms = smem + P.terms;
 
   if (c.warp == 0) {
     tmem_alloc(sp<uint32_t>(S_TMEM), kTmemCols);
@@ -86,7 +86,7 @@ __global__ void __launch_bounds__(kT, 3) k_window(const StepArgs a) {
     const Meta m = *meta;
     const bool valid = m.slot >= 0 && m.slot < a.n_slots;
     const uint32_t kb = (uint32_t)dk * P.esz, vb = (uint32_t)dv * P.esz;
-    const uint32_t ab = GATE == 1 ? 4u * dk : 0u, rb = ROWS ? 4u * dk : 0u, shb = 16u + 4u * dk;
+    const uint32_t ab = GATE == 1 ? 4u * dk : 0u, rb = ROWS ? 4u * dk : 0u, shb = P.side.head;
     if (c.lane == 0) {
       int* nf = flag_base + 4 * fslot;
       nf[F_INPUT] = nf[F_RANGE] = nf[F_UNDER] = 0;
@@ -148,7 +148,7 @@ __global__ void __launch_bounds__(kT, 3) k_window(const StepArgs a) {
       if (cnt > 0)
         bulk_load(terms,
                   a.side + (size_t)hdr.slot * a.side_slot_bytes + (size_t)hdr.h * a.side_head_bytes +
-                      16u + 4u * dk,
+                      P.side.head,
                   (uint32_t)cnt * tbytes, tfull);
     }
     const int io = hdr.b * H + hdr.h;
@@ -178,7 +178,9 @@ __global__ void __launch_bounds__(kT, 3) k_window(const StepArgs a) {
         const float ki = ld_io(st + P.k_off, IO, i), qi = ld_io(st + P.q_off, IO, i);
         const float ai = GATE == 0 ? hdr.alpha : reinterpret_cast<const float*>(st + P.al_off)[i];
         bad_in |= !isfinite(ki) || !isfinite(qi) || !isfinite(ai);
-        const float gold = cnt > 0 ? reinterpret_cast<const float*>(st + P.sh_off + 16)[i] : 1.f;
+        const float gold = cnt == 0 ? 1.f
+                           : GATE == 1 ? reinterpret_cast<const float*>(st + P.sh_off + 16)[i]
+                                       : reinterpret_cast<const float*>(st + P.sh_off)[1];
         const float gn = gold * ai;
         under |= gn < 1e-30f;
         const float yi = gn * ki, zi = gn * qi;
@@ -277,7 +279,8 @@ __global__ void __launch_bounds__(kT, 3) k_window(const StepArgs a) {
       for (int t = c.warp; t < cnt; t += kW) {
         float dy = 0.f, dz = 0.f;
         if (4 * c.lane < dk) {
-          const float4 kh = *reinterpret_cast<const float4*>(terms + (size_t)t * (dk + dv) + 4 * c.lane);
+          const int rows4[4] = {4 * c.lane, 4 * c.lane + 1, 4 * c.lane + 2, 4 * c.lane + 3};
+          const float4 kh = term_k4<GATE == 0 && IO == 1, false>(terms + (size_t)t * tbytes, rows4);
           const float4 y4 = *reinterpret_cast<const float4*>(sp<float>(W_Y) + 4 * c.lane);
           const float4 z4 = *reinterpret_cast<const float4*>(sp<float>(W_Z) + 4 * c.lane);
           dy = __fmaf_rn(kh.x, y4.x, __fmaf_rn(kh.y, y4.y, __fmaf_rn(kh.z, y4.z, kh.w * y4.w)));
@@ -303,12 +306,12 @@ __global__ void __launch_bounds__(kT, 3) k_window(const StepArgs a) {
       // ---- u, b, o of column t ----
       const bool fold = cnt + 1 >= W || c.flags[F_UNDER] != 0;
       uint8_t* side = a.side + (size_t)hdr.slot * a.side_slot_bytes + (size_t)hdr.h * a.side_head_bytes;
-      float* tnew = reinterpret_cast<float*>(side + 16 + 4 * dk) + (size_t)cnt * (dk + dv);
+      uint8_t* tnew = side + P.side.head + (size_t)cnt * tbytes;
       if (tid < dv) {
         float u = u0 + sp<float>(W_OU)[tid], pq = p0 + sp<float>(W_OP)[tid];
         const float2* lr = reinterpret_cast<const float2*>(sp<float>(W_LR));
         for (int t = 0; t < cnt; ++t) {
-          const float bt = terms[(size_t)t * (dk + dv) + dk + tid];
+          const float bt = reinterpret_cast<const float*>(terms + (size_t)t * tbytes + kbytes)[tid];
           const float2 l = lr[t];
           u = __fmaf_rn(l.x, bt, u);
           pq = __fmaf_rn(l.y, bt, pq);
@@ -319,22 +322,34 @@ __global__ void __launch_bounds__(kT, 3) k_window(const StepArgs a) {
         out[tid] = __fmaf_rn(bj, kqv, pq);
         if (fold)
           sp<float>(W_OU)[tid] = bj;  // b for the fold (the column's share of u is used up)
-        else
-          tnew[dk + tid] = bj;
+        else  // the b part: b, or b / g for the scalar gate
+          reinterpret_cast<float*>(tnew + kbytes)[tid] = GATE == 1 ? bj : bj / sp<float>(W_GN)[0];
       }
       if (!fold) {  // append this token's factors, keep the window open
-        if (tid < dk) {
-          tnew[tid] = sp<float>(W_K)[tid] / sp<float>(W_GN)[tid];
-          reinterpret_cast<float*>(side + 16)[tid] = sp<float>(W_GN)[tid];
+        if (GATE == 1) {  // k_hat = k / g and the gates
+          if (tid < dk) {
+            reinterpret_cast<float*>(tnew)[tid] = sp<float>(W_K)[tid] / sp<float>(W_GN)[tid];
+            reinterpret_cast<float*>(side + 16)[tid] = sp<float>(W_GN)[tid];
+          }
+          if (tid == 0) *reinterpret_cast<int32_t*>(side) = cnt + 1;
+        } else {  // the token's k as given (W_K holds it exactly), the gate in the header
+          if (tid < dk) {
+            if (IO == 1)
+              reinterpret_cast<uint16_t*>(tnew)[tid] = (uint16_t)(__float_as_uint(sp<float>(W_K)[tid]) >> 16);
+            else
+              reinterpret_cast<float*>(tnew)[tid] = sp<float>(W_K)[tid];
+          }
+          if (tid == 0)
+            *reinterpret_cast<int2*>(side) = make_int2(cnt + 1, __float_as_int(sp<float>(W_GN)[0]));
         }
-        if (tid == 0) *reinterpret_cast<int32_t*>(side) = cnt + 1;
       } else {  // end of the window: fold everything into the block
         __syncthreads();
         float4 bv = make_float4(0.f, 0.f, 0.f, 0.f);
         if (c.act()) bv = *reinterpret_cast<const float4*>(sp<float>(W_OU) + 4 * c.lane);
         uint8_t* dst = a.pool + (size_t)hdr.slot * a.slot_bytes + hdr.off;
-        window_fold<GATE, FULL, ROWS>(c, a, blk, terms, cnt, mode, cv, bv, dst, omega,
-                                      reinterpret_cast<int32_t*>(side));
+        window_fold<GATE, FULL, ROWS, GATE == 0 && IO == 1>(c, a, blk, terms, tbytes, kbytes, cnt,
+                                                             mode, cv, bv, dst, omega,
+                                                             reinterpret_cast<int32_t*>(side));
       }
     }
     __syncthreads();  // the term buffer and this item's shared arrays are free

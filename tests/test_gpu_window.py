@@ -29,6 +29,7 @@ CASES = {
     "win-d128": W.small("window", batch=2, n_heads=3, d=128).scaled(window=5),
     "win-mixed": W.small("gdn", batch=2, n_heads=4, d=64).scaled(window=3, n_outliers=4),
     "win-kda": W.small("kda", batch=2, n_heads=2, d=32).scaled(window=4, n_outliers=8),
+    "win-f32io": W.small("window", batch=2, n_heads=2, d=64, io_dtype=W.IO_F32).scaled(window=4),
 }
 
 
@@ -76,7 +77,7 @@ def test_window_lockstep(name):
     assert case.pool.status() == (sq.SQ_OK, 0)
 
 
-@pytest.mark.parametrize("name", ["win-s", "win-kda"])
+@pytest.mark.parametrize("name", ["win-s", "win-kda", "win-f32io"])
 def test_window_flush_mid_window(name):
     wl = CASES[name]
     case = G.GpuCase(wl)
