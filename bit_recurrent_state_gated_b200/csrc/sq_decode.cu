@@ -315,39 +315,8 @@ __global__ void __launch_bounds__(kT, kMaxCtasPerSm) k_decode(const StepArgs a) 
       __syncthreads();
       continue;
     }
-    float r = row_scales(c, true, omega);
-    // the second (and last) alternation may be provably unable to change an fp16 scale (see
-    // row_scale_settled); not with row weights, whose closing refit needs the exact fp32 scales
-    const bool may_settle = a.fit_iters == 2 && !a.omega && !a.full_fit;
-    col_pass(c, sp<float>(S_REDC));
-    const bool unsettled_row = __syncthreads_or(may_settle && !row_scale_settled(r));  // barrier 2
-    float4 cm = max4(sp<float>(S_REDC), c.lane);
-    const bool settled =  // the same in every warp: each holds every column scale
-        may_settle && !unsettled_row && __all_sync(0xffffffffu, !c.act() || column_scales_settled(cm));
-    for (int f = 1; f < a.fit_iters && !settled; ++f) {
-      // the last column pass may be skipped (see column_slack); not with row weights, whose
-      // closing refit needs the exact fp32 column scales
-      const bool maybe_skip = f + 1 == a.fit_iters && !a.omega && !a.full_fit;
-      if (maybe_skip) column_slack(c.warp, c.lane, cm, c.act());
-      const float w_old = sp<float>(S_W)[c.row0() + c.lane];
-      row_pass(c, make_float4(rcp_rn(cm.x), rcp_rn(cm.y), rcp_rn(cm.z), rcp_rn(cm.w)));
-      r = row_scales(c, false, omega);
-      if (maybe_skip) {
-        multiplier_change(c.warp, c.lane, w_old, sp<float>(S_W)[c.row0() + c.lane]);
-        __syncthreads();  // barrier 3 (fit_iters = 2): slack and changes of every warp
-        const float4 d4 = *sp<float4>(S_FIT);
-        if (fmaxf(fmaxf(d4.x, d4.y), fmaxf(d4.z, d4.w)) <= sp<float>(S_FIT)[4]) break;
-      }
-      float* red = sp<float>(S_REDC) + (f & 1) * kW * kMaxD;
-      col_pass(c, red);
-      __syncthreads();  // barrier 3 (or 4 after a failed skip test)
-      cm = max4(red, c.lane);
-    }
-    if (a.omega) {  // rows weighted below 1: fit once more against the final column scales
-      row_pass(c, make_float4(rcp_rn(cm.x), rcp_rn(cm.y), rcp_rn(cm.z), rcp_rn(cm.w)));
-      r = row_refit(c, r, omega);
-      __syncthreads();  // every warp sees the range flags the refit may have set
-    }
+    float4 cm;
+    const float r = fit_scales(c, a, omega, cm);
     if (c.flags[F_RANGE]) {
       if (tid == 0) atomicOr(a.flag, SQ_FLAG_RANGE_BIT);
       continue;

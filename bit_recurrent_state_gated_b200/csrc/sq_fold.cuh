@@ -445,23 +445,8 @@ __device__ __forceinline__ void window_fold(const Ctx<FULL>& c, const StepArgs& 
     });
     __syncwarp();
   }
-  float r = row_scales(c, true, omega);
-  col_pass(c, sp<float>(S_REDC));
-  __syncthreads();
-  float4 cm = max4(sp<float>(S_REDC), lane);
-  for (int f = 1; f < a.fit_iters; ++f) {
-    row_pass(c, make_float4(rcp_rn(cm.x), rcp_rn(cm.y), rcp_rn(cm.z), rcp_rn(cm.w)));
-    r = row_scales(c, false, omega);
-    float* red = sp<float>(S_REDC) + (f & 1) * kW * kMaxD;
-    col_pass(c, red);
-    __syncthreads();
-    cm = max4(red, lane);
-  }
-  if (a.omega) {  // rows weighted below 1: fit once more against the final column scales
-    row_pass(c, make_float4(rcp_rn(cm.x), rcp_rn(cm.y), rcp_rn(cm.z), rcp_rn(cm.w)));
-    r = row_refit(c, r, omega);
-    __syncthreads();  // every warp sees the range flags the refit may have set
-  }
+  float4 cm;
+  const float r = fit_scales(c, a, omega, cm);
   if (c.flags[F_RANGE]) {
     if (tid == 0) {
       atomicOr(a.flag, SQ_FLAG_RANGE_BIT);

@@ -586,6 +586,48 @@ __device__ __forceinline__ float4 sum4(const float* red, int lane) {
   return make_float4(x.x, x.y, y.x, y.y);
 }
 
+// The scale fit of an item after the row maxima are in S_RT (all threads; fit_iters
+// alternations of row and column max-abs passes): returns the lane's row scale r and the lane's
+// four column scales in cm, fp32, as the rule computes them, except where the fp16 values
+// provably cannot differ (the two exact shortcuts below). Three CTA barriers for fit_iters = 2.
+template <class C>
+__device__ __forceinline__ float fit_scales(const C& c, const StepArgs& a, float omega, float4& cm) {
+  float r = row_scales(c, true, omega);
+  // the second (and last) alternation may be provably unable to change an fp16 scale (see
+  // row_scale_settled); not with row weights, whose closing refit needs the exact fp32 scales
+  const bool may_settle = a.fit_iters == 2 && !a.omega && !a.full_fit;
+  col_pass(c, sp<float>(S_REDC));
+  const bool unsettled_row = __syncthreads_or(may_settle && !row_scale_settled(r));
+  cm = max4(sp<float>(S_REDC), c.lane);
+  const bool settled =  // the same in every warp: each holds every column scale
+      may_settle && !unsettled_row && __all_sync(0xffffffffu, !c.act() || column_scales_settled(cm));
+  for (int f = 1; f < a.fit_iters && !settled; ++f) {
+    // the last column pass may be skipped (see column_slack); not with row weights
+    const bool maybe_skip = f + 1 == a.fit_iters && !a.omega && !a.full_fit;
+    if (maybe_skip) column_slack(c.warp, c.lane, cm, c.act());
+    const float w_old = sp<float>(S_W)[c.row0() + c.lane];
+    row_pass(c, make_float4(rcp_rn(cm.x), rcp_rn(cm.y), rcp_rn(cm.z), rcp_rn(cm.w)));
+    r = row_scales(c, false, omega);
+    if (maybe_skip) {
+      multiplier_change(c.warp, c.lane, w_old, sp<float>(S_W)[c.row0() + c.lane]);
+      __syncthreads();  // slack and changes of every warp
+      const float4 d4 = *sp<float4>(S_FIT);
+      if (fmaxf(fmaxf(d4.x, d4.y), fmaxf(d4.z, d4.w)) <= sp<float>(S_FIT)[4]) break;
+    }
+    float* red = sp<float>(S_REDC) + (f & 1) * kW * kMaxD;
+    col_pass(c, red);
+    __syncthreads();
+    cm = max4(red, c.lane);
+  }
+  if (a.omega) {  // rows weighted below 1: fit once more against the final column scales
+    row_pass(c, make_float4(rcp_rn(cm.x), rcp_rn(cm.y), rcp_rn(cm.z), rcp_rn(cm.w)));
+    r = row_refit(c, r, omega);
+    __syncthreads();  // every warp sees the range flags the refit may have set
+  }
+  return r;
+}
+
+
 // ---- requantize, pack and store ----------------------------------------------------------
 // Row scales: r16_i to the block (at the original row), t_i / r16_i into S_IR (t_i for fp16
 // rows); column scales: c16.
