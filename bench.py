@@ -27,10 +27,10 @@ times the CPU oracle on a bounded sample of the same workload on the host cores.
 from __future__ import annotations
 
 import argparse
-import glob
 import hashlib
 import json
 import os
+import re
 import statistics
 import sys
 import threading
@@ -109,21 +109,41 @@ def peaks() -> tuple[float, str]:
         return 6650.0, "fallback"
 
 
-def source_digest() -> str:
+# The sources each timed kernel is built from (its translation units, the headers they include
+# and the host code that lays out its tables and launches it).
+_COMMON = ["sq_step.cuh", "sq_pair.cuh", "sq_device.cuh", "sq_tile.cuh", "sq_internal.h",
+           "sq_api.cu"]
+KERNEL_SOURCES = {
+    "k_decode": ["sq_decode.cu"] + _COMMON,
+    "k_window": ["sq_window_step.cu", "sq_fold.cuh"] + _COMMON,
+    "k_chunk": ["sq_chunk.cu", "sq_fold.cuh"] + _COMMON,
+    "k_decode_k_quantize": ["sq_decode.cu", "sq_quant.cu"] + _COMMON,
+}
+
+
+def _code_only(text: str) -> str:
+    """The source without comments and with whitespace collapsed: edits to comments do not
+    change what the kernel computes."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
+def source_digest(kernel: str = "k_decode", root: str = ROOT) -> str:
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "bit_recurrent_state_gated_b200", "csrc", "*"))):
-        with open(p, "rb") as f:
-            h.update(f.read())
+    for name in sorted(KERNEL_SOURCES[kernel]):
+        with open(os.path.join(root, "bit_recurrent_state_gated_b200", "csrc", name)) as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 
 def profiled_traffic(workload: str, kernel: str = "k_decode"):
     """DRAM bytes per launch of the timed kernel from the committed ncu summary, if it was
-    taken on the current kernel source (else None)."""
+    taken on the current source of that kernel (else None)."""
     p = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
     if not os.path.exists(p):
         return None
-    digest = source_digest()
+    digest = source_digest(kernel)
     with open(p) as f:
         for line in f:
             if line.startswith("bench-traffic:"):

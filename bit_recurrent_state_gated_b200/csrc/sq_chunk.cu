@@ -233,7 +233,7 @@ __global__ void __launch_bounds__(kT, ROWS ? 4 : 3) k_chunk(const StepArgs a) {
       *reinterpret_cast<int4*>(shdr) = make_int4(valid, slot, k.b, h);
       *(reinterpret_cast<int4*>(shdr) + 1) =
           make_int4(0, 0, hd.pivot_head ? MODE_PIVOT : (int)hd.width, (int)hd.off);
-      mbar_arrive_expect_tx(full, valid ? 2 * qb + vb + ab + rb + hd.bytes : 0u);
+      mbar_arrive_expect_tx(full, valid ? 2 * qb + vb + ab + rb + hd.bytes + a.extra_tx : 0u);
     }
     if (valid && c.lane >= 1 && c.lane <= 6) {
       uint8_t* dst = s;
@@ -261,9 +261,10 @@ __global__ void __launch_bounds__(kT, ROWS ? 4 : 3) k_chunk(const StepArgs a) {
 
   int it = 0;
   bool timed_out = false;
+  const uint64_t wait_ns = a.wait_ns ? a.wait_ns : kWaitLimitNs;
   int32_t dummy_count = 0;
   for (int item = first; item < n_items; item += stride, ++it) {
-    const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(full, (uint32_t)it & 1u));
+    const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(full, (uint32_t)it & 1u, wait_ns));
     c.flags = flag_base + 4 * (it & 3);
     StageHdr hdr = *reinterpret_cast<const StageHdr*>(st);
     if (!ok) hdr.valid = 0;
@@ -446,7 +447,7 @@ __global__ void __launch_bounds__(kT, ROWS ? 4 : 3) k_chunk(const StepArgs a) {
   }
   if (timed_out) {
     if (tid == 0) atomicOr(a.flag, SQ_FLAG_TIMEOUT_BIT);
-    mbar_wait_bounded(full, (uint32_t)it & 1u);  // the copy in flight, if any
+    mbar_wait_bounded(full, (uint32_t)it & 1u, wait_ns);  // the copy in flight, if any
     if (producer && c.lane < 32) cp_async_wait_all();
   }
   tmem_fence_before_sync();

@@ -23,16 +23,16 @@ namespace {
 // the per-step kernel's fit and requantize passes on the rest.
 //
 // Side block of one (slot, head): see SideFmt (sq_internal.h); for the scalar gate a term holds
-// the token's k in the I/O type and b_s / g_s, whose product is k_hat_s b_s^T. Two stages hold
-// the next items' q, k, v (alpha, row table), side header (+ g) and frozen block; the low-rank
-// terms, whose count is known only once the header has landed, follow into their own buffer
-// while pass A runs.
+// the token's k in the I/O type and b_s / g_s, whose product is k_hat_s b_s^T. The staging
+// buffer holds the next item's q, k, v (alpha, row table), side header (+ g) and frozen block;
+// the low-rank terms, whose count is known only once the header has landed, follow into their
+// own buffer while pass A runs.
 // =============================================================================================
 constexpr int kMaxWin = 64;
 constexpr int kMaxCand = 256;  // candidate entries for the compensation choice
 
 // Window-only shared memory, after the per-step kernel's fixed arrays.
-constexpr uint32_t W_BAR = S_STAGE;          // full[2], tfull
+constexpr uint32_t W_BAR = S_STAGE;          // full (stage), tfull (terms)
 constexpr uint32_t W_Y = W_BAR + 32;         // y, z, k, g by original row
 constexpr uint32_t W_Z = W_Y + 512;
 constexpr uint32_t W_K = W_Z + 512;
@@ -47,7 +47,7 @@ constexpr uint32_t W_OIDX = W_TKEY + 512;    // chosen entries: flat index, posi
 constexpr uint32_t W_OPOS = W_OIDX + 256;
 constexpr uint32_t W_OVAL = W_OPOS + 256;
 constexpr uint32_t W_MISC = W_OVAL + 256;    // [0] candidates, [1] threshold key, [2] entries'
-                                             // byte offset, [4..5] items issued per stage
+                                             // byte offset, [4] items staged
 constexpr uint32_t W_OE = W_MISC + 64;       // the frozen block's compensation entries:
                                              // flat index [64] int, value [64] float
 constexpr uint32_t W_STAGE = W_OE + 512;
@@ -59,8 +59,8 @@ static_assert(12 * kMaxCand + 3 * 64 * 4 <= 4096, "candidates fit the column-max
 
 enum { F_UNDER = 2 };
 
-// Stage: header, k, q, v, (alpha), (row table), side header + g, block; two stages, then the
-// low-rank term buffer and the head table.
+// Stage: header, k, q, v, (alpha), (row table), side header (+ g), block; then the low-rank term
+// buffer and the head table.
 struct WDPlan {
   uint32_t esz, k_off, q_off, v_off, al_off, rt_off, sh_off, blk_off, stage, terms, tab, total;
   SideFmt side;
@@ -76,7 +76,7 @@ struct WDPlan {
     sh_off = rt_off + (per_row ? 4u * dk : 0u);
     blk_off = sh_off + side.head;
     stage = blk_off + round16(stage_bytes + kSlack);
-    terms = W_STAGE + 2u * stage;
+    terms = W_STAGE + stage;
     tab = terms + (uint32_t)(window - 1) * side.stride;
     total = tab + round16(20u * (uint32_t)n_heads);
   }

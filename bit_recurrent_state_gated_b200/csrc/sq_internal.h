@@ -82,8 +82,9 @@ struct StepArgs {
   int32_t update_only;  // with s_new: write the updated fp32 state and stop (no refit, no
                         // requantization); a skipped item gets a NaN in its s_new block
   uint64_t wait_ns;     // limit of every wait on a bulk copy (global-timer nanoseconds)
-  uint32_t extra_tx;    // test hook: bytes the decode kernel's stage barrier expects beyond
-                        // what its copies bring (0 in normal use; > 0 makes the wait run out)
+  uint32_t extra_tx;    // test hook: bytes the staging barrier of the decode, window and chunk
+                        // kernels expects beyond what its copies bring (0 in normal use; > 0
+                        // makes the wait run out)
   int32_t full_fit;     // test hook: 1 = never skip the last column pass of the fit
 };
 

@@ -5,11 +5,16 @@
 namespace sq {
 namespace {
 
+// One staging buffer, refilled with the next item right after the current item's first barrier
+// (as in the decode kernel): with the term buffer that keeps a CTA within a quarter of the SM's
+// shared memory and 128 registers, so four CTAs (sixteen warps) share an SM. The in-window token
+// is bound by latency, not by issue, so the extra warps matter more than the shorter lead of the
+// copies (two staging buffers at three CTAs per SM: 75 us per in-window token at 256 x 32).
 template <int GATE, int IO, bool FULL, bool ROWS>
-__global__ void __launch_bounds__(kT, 3) k_window(const StepArgs a) {
+__global__ void __launch_bounds__(kT, 4) k_window(const StepArgs a) {
   const WDPlan P(a.dk, a.dv, IO, GATE, ROWS, a.stage_bytes, a.H, a.window);
   uint64_t* full = sp<uint64_t>(W_BAR);
-  uint64_t* tfull = full + 2;
+  uint64_t* tfull = full + 1;
   Ctx<FULL> c;
   c.tid = threadIdx.x;
   c.warp = c.tid >> 5;
@@ -32,7 +37,7 @@ __global__ void __launch_bounds__(kT, 3) k_window(const StepArgs a) {
     tmem_relinquish();
   }
   if (tid == 0) {
-    for (int s = 0; s < 3; ++s) mbar_init(&full[s], 1);
+    for (int s = 0; s < 2; ++s) mbar_init(&full[s], 1);
     fence_mbar_init();
   }
   if (tid < 16) sp<int>(S_FLAGS)[tid] = 0;
@@ -96,7 +101,7 @@ __global__ void __launch_bounds__(kT, 3) k_window(const StepArgs a) {
       *(reinterpret_cast<int4*>(shdr) + 1) =
           make_int4(__float_as_int(m.beta), __float_as_int(GATE == 0 ? m.alpha : 0.f),
                     hd.pivot_head ? MODE_PIVOT : (int)hd.width, (int)hd.off);
-      mbar_arrive_expect_tx(&full[s], valid ? 2 * kb + vb + ab + rb + shb + hd.bytes : 0u);
+      mbar_arrive_expect_tx(&full[s], valid ? 2 * kb + vb + ab + rb + shb + hd.bytes + a.extra_tx : 0u);
     }
     if (valid && c.lane >= 1 && c.lane <= 7) {
       uint8_t* dst = st;
@@ -121,23 +126,24 @@ __global__ void __launch_bounds__(kT, 3) k_window(const StepArgs a) {
     advance(k);
   };
 
-  if (tid == 0) sp<int>(W_MISC)[4] = sp<int>(W_MISC)[5] = 0;
+  if (tid == 0) sp<int>(W_MISC)[4] = 0;
   __syncthreads();
   if (producer) {
     fetch_meta(next_meta);
-    for (int s = 0; s < 2 && next_issue.item < n_items; ++s) {
-      issue(next_issue, s, s);
+    if (next_issue.item < n_items) {
+      issue(next_issue, 0, 0);
       fetch_meta(next_meta);
     }
   }
 
   int it = 0;
   bool timed_out = false;
+  const uint64_t wait_ns = a.wait_ns ? a.wait_ns : kWaitLimitNs;
   for (int item = first; item < n_items; item += stride, ++it) {
-    const int s = it & 1;
-    const uint8_t* st = smem + W_STAGE + s * P.stage;
+    const int s = 0;
+    const uint8_t* st = smem + W_STAGE;
     const uint8_t* blk = st + P.blk_off;
-    const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&full[s], (uint32_t)(it >> 1) & 1u));
+    const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&full[s], (uint32_t)it & 1u, wait_ns));
     c.flags = flag_base + 4 * (it & 3);
     StageHdr hdr = *reinterpret_cast<const StageHdr*>(st);
     if (!ok) hdr.valid = 0;
@@ -260,9 +266,9 @@ __global__ void __launch_bounds__(kT, 3) k_window(const StepArgs a) {
       u0 = tc * ((ru[0] + ru[kMaxD]) + (ru[2 * kMaxD] + ru[3 * kMaxD]));
       p0 = tc * ((rp[0] + rp[kMaxD]) + (rp[2 * kMaxD] + rp[3 * kMaxD]));
     }
-    // the frozen block is no longer read: stage the item after next into its buffer
+    // the stage is no longer read: stage the next item
     if (producer && next_issue.item < n_items) {
-      issue(next_issue, s, (it + 2) & 3);
+      issue(next_issue, s, (it + 1) & 3);
       fetch_meta(next_meta);
     }
     // frozen compensation entries' share of u and o
@@ -274,7 +280,7 @@ __global__ void __launch_bounds__(kT, 3) k_window(const StepArgs a) {
         atomicAdd(sp<float>(W_OP) + idx % dv, pv * sp<float>(W_Z)[idx / dv]);
       }
     }
-    const bool tok = __all_sync(0xffffffffu, mbar_wait_bounded(tfull, (uint32_t)it & 1u));
+    const bool tok = __all_sync(0xffffffffu, mbar_wait_bounded(tfull, (uint32_t)it & 1u, wait_ns));
     if (!skip) {  // low-rank coefficients, one term per warp at a time
       for (int t = c.warp; t < cnt; t += kW) {
         float dy = 0.f, dz = 0.f;
@@ -357,14 +363,11 @@ __global__ void __launch_bounds__(kT, 3) k_window(const StepArgs a) {
 
   if (timed_out) {
     if (tid == 0) atomicOr(a.flag, SQ_FLAG_TIMEOUT_BIT);
-    // let copies still in flight land before the CTA exits: stage s has received
-    // W_MISC[4 + s] copies, of which the items before `it` consumed (it + 1 - s) / 2
+    // let copies still in flight land before the CTA exits: the stage has received W_MISC[4]
+    // copies, of which the items before `it` consumed `it`
     __syncthreads();
-    for (int s2 = 0; s2 < 2; ++s2) {
-      const int issued = sp<int>(W_MISC)[4 + s2], used = (it + 1 - s2) / 2;
-      for (int u = used; u < issued; ++u) mbar_wait_bounded(&full[s2], (uint32_t)u & 1u);
-    }
-    mbar_wait_bounded(tfull, (uint32_t)it & 1u);
+    for (int u = it; u < sp<int>(W_MISC)[4]; ++u) mbar_wait_bounded(&full[0], (uint32_t)u & 1u, wait_ns);
+    mbar_wait_bounded(tfull, (uint32_t)it & 1u, wait_ns);
     if (producer && c.lane < 3) cp_async_wait_all();
   }
   tmem_fence_before_sync();

@@ -275,14 +275,15 @@ SQ_API sq_status sq_debug_decode_step_fp32(sq_pool* pool, const int32_t* slot_id
 
 /*
  * Test hook for the bounded waits (the pages have no counterpart: it exists so that the
- * timeout path can be exercised without faulting anything). Every later sq_decode_step and
- * sq_debug_decode_step_fp32 on this pool (window == 1) gives up a wait on a bulk copy after
+ * timeout path can be exercised without faulting anything). Every later sq_decode_step (the
+ * per-step and the windowed kernel), sq_decode_chunk and sq_debug_decode_step_fp32 on this pool
+ * gives up a wait on a bulk copy after
  * wait_limit_ns nanoseconds of the GPU's global timer (0 restores the default, 1 s), and, with
  * extra_expected_bytes > 0 (at most 4096), has each copy's barrier expect that many bytes more
  * than the copies bring, so that every wait runs out. A kernel whose wait runs out sets
  * SQ_FLAG_TIMEOUT (sq_pool_status then returns SQ_ERR_TIMEOUT), lets its own copies land, frees
- * its tensor memory and returns; the items it did not reach keep their slot bytes and their
- * output rows are not written. Host only; nothing is enqueued. Call with 0, 0 to restore normal
+ * its tensor memory and returns; the items it did not reach keep their slot bytes (and their
+ * window side state) and their output rows are not written. Host only; nothing is enqueued. Call with 0, 0 to restore normal
  * operation. SQ_ERR_INVALID_ARG for a NULL pool or more than 4096 extra bytes. */
 SQ_API sq_status sq_debug_set_wait(sq_pool* pool, uint64_t wait_limit_ns,
                                    uint32_t extra_expected_bytes);
