@@ -61,6 +61,9 @@ def parse():
                                                           "chunk", "split"])
     ap.add_argument("--runs", type=int, default=5, help="timed regions of K steps (median)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cold-window", action="store_true",
+                    help="windowed workloads: run one whole window after the cold quantize, "
+                         "untimed, and exit (a fixed launch sequence for the profiler)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
     return ap.parse_args()
@@ -270,6 +273,27 @@ def oracle_rate(wl: W.Workload, seconds: float, t0: int = 0):
 
 # ---- GPU arm -----------------------------------------------------------------------------------
 
+def cold_window(wl, pool, si):
+    """W tokens from the cold start (W - 1 in-window tokens, then the fold), untimed."""
+    import torch
+    if wl.window <= 1:
+        raise SystemExit("--cold-window needs a windowed workload")
+    out = torch.empty((wl.batch, wl.n_heads, wl.d_v), dtype=torch.float32, device="cuda")
+    for t in range(wl.window):
+        x = wl.step_inputs(t)
+        if wl.io_dtype == W.IO_BF16:
+            q, k, v = (torch.from_numpy(x[n + "_bf16"]).view(torch.bfloat16).cuda() for n in "qkv")
+        else:
+            q, k, v = (torch.from_numpy(x[n]).cuda() for n in "qkv")
+        pool.decode_step(si, q, k, v, torch.from_numpy(x["alpha"]).cuda(),
+                         torch.from_numpy(x["beta"]).cuda(), out)
+    torch.cuda.synchronize()
+    st, flag = pool.status()
+    if st != 0:
+        raise RuntimeError(f"device flag {flag}")
+    return None
+
+
 def run_ours(args, info):
     import torch
 
@@ -288,6 +312,8 @@ def run_ours(args, info):
     for c in range(0, wl.batch, 64):  # initial states, quantized on the GPU in chunks
         S0 = torch.from_numpy(wl.initial_state(si_np[c:c + 64])).cuda()
         pool.quantize(si[c:c + 64], S0)
+    if args.cold_window:
+        return cold_window(wl, pool, si)
     T = wl.tokens
     n_sets = max(1, min(args.steps + args.warmup, 8))
     sets_host, sets_dev = [], []
