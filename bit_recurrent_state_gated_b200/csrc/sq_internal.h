@@ -106,7 +106,8 @@ struct QuantArgs {
   int64_t side_slot_bytes, side_head_bytes;
 };
 
-// Launchers (sq_decode.cu, sq_quant.cu, sq_window.cu). Return cudaSuccess or the launch error.
+// Launchers (sq_decode.cu, sq_quant.cu, sq_window_step.cu, sq_window.cu, sq_chunk.cu). Return
+// cudaSuccess or the launch error.
 cudaError_t launch_decode(const StepArgs& a, int gate, int io, bool want_state, int num_sms,
                           cudaStream_t st);
 cudaError_t launch_quantize(const QuantArgs& a, cudaStream_t st);
