@@ -30,6 +30,7 @@ CASES = {
     "kda-d64": W.small("kda", batch=2, n_heads=2, d=64),
     "kda-d128": W.small("kda", batch=2, n_heads=2, d=128),
     "pool-d96": W.small("pool", batch=3, n_heads=3, d=96),
+    "kda-pivots": W.small("kda", batch=2, n_heads=2, d=64, n_pivots=32),
     "tiny": W.WORKLOADS["tiny"],
 }
 

@@ -36,6 +36,8 @@ def small_cases():
         "gdn-fit1": W.small("gdn", batch=2, n_heads=4, d=64, fit_iters=1),
         "gdn-f32io": W.small("gdn", batch=2, n_heads=4, d=64, io_dtype=W.IO_F32),
         "kda-many": W.small("kda", batch=40, n_heads=16, d=32),  # > 2 items per CTA, ragged
+        # a quarter of the key rows fp16: whole four-row chunks of fp16 rows (their own path)
+        "kda-pivots": W.small("kda", batch=3, n_heads=2, d=64, n_pivots=32),
     }
 
 

@@ -30,6 +30,8 @@ CASES = {
     "win-mixed": W.small("gdn", batch=2, n_heads=4, d=64).scaled(window=3, n_outliers=4),
     "win-kda": W.small("kda", batch=2, n_heads=2, d=32).scaled(window=4, n_outliers=8),
     "win-f32io": W.small("window", batch=2, n_heads=2, d=64, io_dtype=W.IO_F32).scaled(window=4),
+    "win-kda-pivots": W.small("kda", batch=2, n_heads=2, d=64, n_pivots=32).scaled(window=4,
+                                                                                 n_outliers=8),
 }
 
 
