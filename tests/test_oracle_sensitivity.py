@@ -2,7 +2,7 @@
 packed start whose inputs differ by one ulp of v at every step (a rounding-level difference,
 smaller than the one between the GPU's fp32 update and the oracle's fp64 one) part ways. Each
 1-LSB code flip moves an element by a whole quantization step, and the next updates spread it,
-so the fraction of equal codes falls step by step. The GPU tests therefore judge parity in
+so the fraction of equal codes falls step by step. The GPU tests therefore check parity in
 lockstep (the oracle restarted from the GPU's bytes every step) and report the free-running
 agreement separately (tests/test_gpu_rollout.py)."""
 import numpy as np
