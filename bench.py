@@ -333,12 +333,13 @@ def run_ours(args, info):
     if args.cold_window:
         return cold_window(wl, pool, si)
     horizon = rollout_calls(wl)
-    since = [0]  # calls on the pool since its last restart
+    since = [0, 0]  # calls on the pool since its last restart; restarts so far
 
     def maybe_restart():  # untimed, like the L2 flush
         if since[0] == horizon:
             restart(pool, si)
             since[0] = 0
+            since[1] += 1
         since[0] += 1
     T = wl.tokens
     n_sets = max(1, min(args.steps + args.warmup, 8))
@@ -407,7 +408,9 @@ def run_ours(args, info):
     runs = max(1, args.runs)
     run_ms, run_kernel_ms = [], []
     with ClockSampler(dev, period_s=0.0005) as clocks:
+        run_restarts = []
         for r in range(runs):
+            restarts0 = since[1]
             ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                   for _ in range(args.steps)]
             dist.barrier()
@@ -422,6 +425,7 @@ def run_ours(args, info):
             dist.barrier()
             kms = [a.elapsed_time(b) for a, b in ev]
             run_kernel_ms.append(kms)
+            run_restarts.append(since[1] - restarts0)
             run_ms.append(dist.max_over_ranks(sum(kms), device="cuda"))
     st, flag = pool.status()
     if st != sq.SQ_OK:
@@ -568,7 +572,11 @@ def run_ours(args, info):
                       f"({n_rot * state_set / 2**20:.0f} MiB of state)",
                 "copies": "own streams, double-buffered (inputs of step t+1 and o of step t "
                           "cross while step t / t+1 computes)"},
-        "gpu_launches": args.steps * (2 if wl.side_stream else 1),  # per timed region
+        # per timed region: the steps' kernels, and the quantize launches of any restart between
+        # steps (outside the steps' events)
+        "gpu_launches": args.steps * (2 if wl.side_stream else 1)
+        + run_restarts[med] * len(range(0, wl.batch, 64)),
+        "rollout": {"restart_every_calls": horizon, "restarts_in_reported_region": run_restarts[med]},
         "clocks": clocks.summary(),
     }
     log("end-to-end region done")
