@@ -412,25 +412,32 @@ __device__ __forceinline__ void pass_b(const C& c, const float4& cv, const float
 // omega: this row's weight in the column passes, in (0, 1] (1 without an impact table): a row
 // weighted below 1 counts with w = fl(omega fl(1 / (r Q))), so it sets the column scales less.
 template <class C>
+__device__ __forceinline__ float row_scale_of(const C& c, int p, float tile_max, bool check,
+                                              float omega, float& w) {
+  float r = 0.f;
+  w = 0.f;
+  const int b = rd_width(sp<uint32_t>(S_RD)[p]);
+  if (b != 16) {
+    const float Q = (float)q_of_width(b);
+    const float inv_q = b == 2 ? 1.0f : b == 4 ? 1.0f / 7.0f : b == 6 ? 1.0f / 31.0f : 1.0f / 127.0f;
+    const float t = sp<float>(S_TR)[p];
+    const float rq = div_q(__fmul_rn(t, tile_max), Q, inv_q);  // exactly m / Q
+    if (check && !(rq < 65520.f)) atomicOr(&c.flags[F_RANGE], 1);
+    r = fminf(fmaxf(rq, kScaleFloor), 65504.f);
+    float wi = rcp_rn(__fmul_rn(r, Q));
+    if (omega < 1.f) wi = __fmul_rn(omega, wi);
+    w = __fmul_rn(t, wi);
+  } else if (check && !(__fmul_rn(sp<float>(S_TR)[p], tile_max) < 65520.f)) {
+    atomicOr(&c.flags[F_RANGE], 1);
+  }
+  return r;
+}
+
+template <class C>
 __device__ __forceinline__ float row_scales(const C& c, bool check, float omega) {
   const int p = c.row0() + c.lane;
   float r = 0.f, w = 0.f;
-  if (p < c.dk()) {
-    const int b = rd_width(sp<uint32_t>(S_RD)[p]);
-    if (b != 16) {
-      const float Q = (float)q_of_width(b);
-      const float inv_q = b == 2 ? 1.0f : b == 4 ? 1.0f / 7.0f : b == 6 ? 1.0f / 31.0f : 1.0f / 127.0f;
-      const float t = sp<float>(S_TR)[p];
-      const float rq = div_q(__fmul_rn(t, sp<float>(S_RT)[p]), Q, inv_q);  // exactly m / Q
-      if (check && !(rq < 65520.f)) atomicOr(&c.flags[F_RANGE], 1);
-      r = fminf(fmaxf(rq, kScaleFloor), 65504.f);
-      float wi = rcp_rn(__fmul_rn(r, Q));
-      if (omega < 1.f) wi = __fmul_rn(omega, wi);
-      w = __fmul_rn(t, wi);
-    } else if (check && !(__fmul_rn(sp<float>(S_TR)[p], sp<float>(S_RT)[p]) < 65520.f)) {
-      atomicOr(&c.flags[F_RANGE], 1);
-    }
-  }
+  if (p < c.dk()) r = row_scale_of(c, p, sp<float>(S_RT)[p], check, omega, w);
   sp<float>(S_W)[p] = w;
   __syncwarp();
   return r;
@@ -586,10 +593,46 @@ __device__ __forceinline__ float4 sum4(const float* red, int lane) {
   return make_float4(x.x, x.y, y.x, y.y);
 }
 
+// The second row pass for those rows of the warp whose scale lies within the margin of an fp16
+// rounding boundary (row_scale_settled), taken as row_pass and row_scales take it: the row's
+// maximum of fl(|T_ij| fl(1/c_j)) over its columns (the chunk holding the row loaded from tensor
+// memory, the lane's four columns, then the warp), then its scale. When every column scale is
+// settled, these are the only scales the second alternation can change. Returns the lane's r.
+template <class C>
+__device__ __forceinline__ float refit_unsettled_rows(const C& c, const float4& cm, float r) {
+  const float ic[4] = {rcp_rn(cm.x), rcp_rn(cm.y), rcp_rn(cm.z), rcp_rn(cm.w)};
+  const int p0 = c.row0();
+  unsigned m = __ballot_sync(0xffffffffu, p0 + c.lane < c.dk() && !row_scale_settled(r));
+  while (m) {
+    const int l = __ffs(m) - 1;  // the row's lane in the warp
+    m &= m - 1;
+    uint32_t regs[16];
+    float2 v[8];
+    tm_issue(c.tm + 16u * (uint32_t)(l >> 2), regs);
+    tm_take(regs, v);
+    // the row's four values by selects on fixed indices (an index computed at run time would
+    // move v to local memory)
+    const bool second_pair = (l >> 1) & 1, odd = l & 1;
+    float mx = 0.f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 g = second_pair ? v[4 + e] : v[e];
+      mx = fmaxf(mx, fabsf(__fmul_rn(odd ? g.y : g.x, ic[e])));
+    }
+    mx = warp_max_nonneg(mx);
+    if (c.lane == l) {
+      float w;
+      r = row_scale_of(c, p0 + l, mx, false, 1.f, w);
+    }
+  }
+  return r;
+}
+
 // The scale fit of an item after the row maxima are in S_RT (all threads; fit_iters
 // alternations of row and column max-abs passes): returns the lane's row scale r and the lane's
 // four column scales in cm, fp32, as the rule computes them, except where the fp16 values
-// provably cannot differ (the two exact shortcuts below). Three CTA barriers for fit_iters = 2.
+// provably cannot differ (the exact shortcuts below). Two or three CTA barriers for
+// fit_iters = 2.
 template <class C>
 __device__ __forceinline__ float fit_scales(const C& c, const StepArgs& a, float omega, float4& cm) {
   float r = row_scales(c, true, omega);
@@ -599,9 +642,12 @@ __device__ __forceinline__ float fit_scales(const C& c, const StepArgs& a, float
   col_pass(c, sp<float>(S_REDC));
   const bool unsettled_row = __syncthreads_or(may_settle && !row_scale_settled(r));
   cm = max4(sp<float>(S_REDC), c.lane);
-  const bool settled =  // the same in every warp: each holds every column scale
-      may_settle && !unsettled_row && __all_sync(0xffffffffu, !c.act() || column_scales_settled(cm));
-  for (int f = 1; f < a.fit_iters && !settled; ++f) {
+  const bool columns_settled =  // the same in every warp: each holds every column scale
+      may_settle && __all_sync(0xffffffffu, !c.act() || column_scales_settled(cm));
+  // with every column scale settled, only the rows near an fp16 boundary can change: their
+  // second row pass alone, row by row (no barrier)
+  if (columns_settled) return unsettled_row ? refit_unsettled_rows(c, cm, r) : r;
+  for (int f = 1; f < a.fit_iters; ++f) {
     // the last column pass may be skipped (see column_slack); not with row weights
     const bool maybe_skip = f + 1 == a.fit_iters && !a.omega && !a.full_fit;
     if (maybe_skip) column_slack(c.warp, c.lane, cm, c.act());
