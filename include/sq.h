@@ -25,6 +25,9 @@
  *   - Within one call every slot index must be distinct; duplicates are not detected and give
  *     an undefined result. Calls on one pool must not overlap in time on different streams
  *     (the second stream of sq_decode_step_split is ordered by the pool itself).
+ *   - A pool lives on the device that was current when it was created, and every later call
+ *     on it must be made with that device current: the library never switches devices, and
+ *     every pointer passed with a pool must be memory of that device.
  *   - State layout: S[i][j] with i the key channel ("key row", [SQ-E] fitting paragraph) and
  *     j the value channel ("value column", [SQ-N]). Dense fp32 states are row-major
  *     [n][n_heads][d_k][d_v].
