@@ -191,11 +191,11 @@ SQ_API sq_status sq_decode_step_split(sq_pool* pool, const int32_t* slot_idx, in
  * Both halves (update, then refit + requantize) run on `stream`. Every call looks up the
  * array's device address on the current device (no address is cached, so a context torn down
  * and created again is harmless); the first call on a device may load the library's module
- * there, so make that first call before any stream capture. All calls in the process share the one array and it keeps the
- * last call's contents (nothing in it needs to start at zero: each call writes every tile it
- * reads back); calls that can run at the same time on the GPU (different streams, different
- * pools) race on it and must be ordered by the caller. Other arguments and errors as
- * sq_decode_step_split. */
+ * there, so make that first call before any stream capture. All calls in the process share
+ * the one array and it keeps the last call's contents (nothing in it needs to start at zero:
+ * each call writes every tile it reads back); calls that can run at the same time on the GPU
+ * (different streams, different pools) race on it and must be ordered by the caller. Other
+ * arguments and errors as sq_decode_step_split. */
 SQ_API sq_status sq_decode_step_split_static(sq_pool* pool, const int32_t* slot_idx,
                                              int32_t batch, const void* q, const void* k,
                                              const void* v, const float* alpha,
